@@ -1,0 +1,183 @@
+"""CPU oracle of the page indexer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+and reference legs may import this package.  The product path
+(``page_scoring_top_b200``) never imports it, and this package imports nothing
+from the product: the two meet only at the seeded inputs.
+
+The arithmetic lives in ``oracle.c`` (plain C, single-threaded, double
+precision, explicit loops, a library sort); this module only compiles it with
+gcc, marshals numpy arrays into it, and states the two acceptance measures the
+pages name:
+
+* the score bound ``|s_gpu - S| <= 1e-5 * A`` per valid entry, with S the exact
+  (double) score and A = sum_h sum_d |q_hd * c_pd| its scale;
+* recall@m ("Iterate Topk", benchmark protocol: recall is reported at
+  floor(3K/4) and at K) = |GPU top-m  intersect  oracle top-m| / min(m, #selectable).
+
+Every function states the passage of the pages it follows in ``oracle.c``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+SCORE_REL_BOUND = 1e-5  # |s_gpu - S| <= SCORE_REL_BOUND * A, per entry
+
+
+def build(force: bool = False) -> str:
+    """Compile ``oracle.c`` into ``liboracle.so`` (gcc, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+             "-fPIC", "-shared", "-fvisibility=hidden", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        L = ctypes.c_int64
+        lib.oracle_scores.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
+        lib.oracle_scores_at.argtypes = [P, P, I, I, I, I, I, L, L, P, P, P, P, P]
+        lib.oracle_topk_f64.argtypes = [P, I, I, P, P]
+        lib.oracle_topk_f32.argtypes = [P, I, I, P, P]
+        lib.oracle_topk_rows_f32.argtypes = [P, P, I, I, L, I, P, P]
+        lib.oracle_topk_rows_f64.argtypes = [P, P, I, I, L, I, P, P]
+        for f in ("oracle_scores", "oracle_scores_at", "oracle_topk_f64", "oracle_topk_f32",
+                  "oracle_topk_rows_f32", "oracle_topk_rows_f64"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def scores(q_bits, c_bits, lengths=None):
+    """Exact scores S and bound scales A, both double [B][T][N].
+
+    ``q_bits``: uint16 bf16 patterns [B][T][Q][D]; ``c_bits``: uint16 [B][N][D];
+    ``lengths``: int32 [B] in [0, N] or None (all valid).
+    """
+    q = _c(q_bits, np.uint16)
+    c = _c(c_bits, np.uint16)
+    B, T, Q, D = q.shape
+    Bc, N, Dc = c.shape
+    assert Bc == B and Dc == D
+    ln = None if lengths is None else _c(lengths, np.int32)
+    S = np.empty((B, T, N), np.float64)
+    A = np.empty((B, T, N), np.float64)
+    rc = _load().oracle_scores(_ptr(q), _ptr(c), _ptr(ln), B, T, Q, D, N, N * D, _ptr(S), _ptr(A))
+    if rc != 0:
+        raise ValueError("oracle_scores: arguments outside the contract")
+    return S, A
+
+
+def scores_at(q_bits, c_bits, b, t, p):
+    """Exact S and A at the listed (b, t, p) triples (spot checks at full size)."""
+    q = _c(q_bits, np.uint16)
+    c = _c(c_bits, np.uint16)
+    B, T, Q, D = q.shape
+    _, N, _ = c.shape
+    b = _c(b, np.int32)
+    t = _c(t, np.int32)
+    p = _c(p, np.int32)
+    n = b.size
+    S = np.empty(n, np.float64)
+    A = np.empty(n, np.float64)
+    rc = _load().oracle_scores_at(_ptr(q), _ptr(c), B, T, Q, D, N, N * D, n,
+                                  _ptr(b), _ptr(t), _ptr(p), _ptr(S), _ptr(A))
+    if rc != 0:
+        raise ValueError("oracle_scores_at: arguments outside the contract")
+    return S, A
+
+
+def topk(row, K, length=None):
+    """Top-K of one row (float32 or float64).  Returns (idx int32[K], val[K], K')."""
+    row = np.asarray(row)
+    n = row.shape[0] if length is None else int(length)
+    idx = np.empty(K, np.int32)
+    if row.dtype == np.float32:
+        r = _c(row, np.float32)
+        val = np.empty(K, np.float32)
+        kk = _load().oracle_topk_f32(_ptr(r), n, K, _ptr(idx), _ptr(val))
+    else:
+        r = _c(row, np.float64)
+        val = np.empty(K, np.float64)
+        kk = _load().oracle_topk_f64(_ptr(r), n, K, _ptr(idx), _ptr(val))
+    if kk < 0:
+        raise ValueError("oracle_topk: arguments outside the contract")
+    return idx, val, kk
+
+
+def topk_rows(scores_2d, K, lengths=None):
+    """Top-K of every row of a [rows][N] array; lengths per row or None."""
+    s = np.asarray(scores_2d)
+    rows, N = s.shape
+    ln = None if lengths is None else _c(lengths, np.int32)
+    idx = np.empty((rows, K), np.int32)
+    if s.dtype == np.float32:
+        s = _c(s, np.float32)
+        val = np.empty((rows, K), np.float32)
+        rc = _load().oracle_topk_rows_f32(_ptr(s), _ptr(ln), rows, N, N, K, _ptr(idx), _ptr(val))
+    else:
+        s = _c(s, np.float64)
+        val = np.empty((rows, K), np.float64)
+        rc = _load().oracle_topk_rows_f64(_ptr(s), _ptr(ln), rows, N, N, K, _ptr(idx), _ptr(val))
+    if rc != 0:
+        raise ValueError("oracle_topk_rows: arguments outside the contract")
+    return idx, val
+
+
+def score_bound_violations(s_gpu, S, A, rel=SCORE_REL_BOUND):
+    """Number of entries breaking the score bound.
+
+    Valid entries (S finite) need |s_gpu - S| <= rel * A; padded entries
+    (S == -inf) need s_gpu == -inf exactly.
+    """
+    s_gpu = np.asarray(s_gpu, np.float64)
+    S = np.asarray(S, np.float64)
+    A = np.asarray(A, np.float64)
+    pad = np.isneginf(S)
+    bad_pad = np.count_nonzero(pad & ~np.isneginf(s_gpu))
+    with np.errstate(invalid="ignore"):
+        err = np.abs(s_gpu - S)
+    bad_val = np.count_nonzero(~pad & ~(err <= rel * A))
+    return int(bad_pad + bad_val)
+
+
+def recall(gpu_idx, oracle_idx, m):
+    """recall@m of one row: |GPU top-m & oracle top-m| / min(m, #selectable).
+
+    Both inputs are index lists in rank order, padded with -1 past K'.
+    Returns 1.0 when nothing is selectable.
+    """
+    g = np.asarray(gpu_idx)[:m]
+    o = np.asarray(oracle_idx)[:m]
+    o = o[o >= 0]
+    g = g[g >= 0]
+    if o.size == 0:
+        return 1.0
+    return np.intersect1d(g, o).size / float(o.size)

@@ -1,0 +1,225 @@
+/*
+ * oracle.c -- plain, slow, single-threaded CPU oracle of the page indexer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or
+ * calls this file: only the tests, the smoke check and the benchmark's
+ * CPU-baseline / reference legs do.  It shares no code, header, table or
+ * helper with the CUDA library; the two meet only at the seeded inputs.
+ *
+ * What it computes, and which passage of the pages defines it
+ * ------------------------------------------------------------
+ * score   "Iterate Centroids Score" (opening description): the indexer scores
+ *         each request's candidate pages from a batch of Q query rows and a
+ *         table of block centroids.  "Round 18 Track C: qsa_topk2 ... +
+ *         qsa_score Query Hoisting & Unrolling", section 1, Target 2, shows
+ *         the per-page score as an FMA reduction over the query heads and the
+ *         head dimension, i.e.
+ *              s[b,t,p] = sum_{h<Q} sum_{d<D} q[b,t,h,d] * c[b,p,d].
+ *         "Round 15 Track C Audit", section 1, Target 1 item 3, scores a tile
+ *         of 16 query tokens at once (the T > 1 prefill-chunk case).
+ *         Pages p >= len[b] are padding and score -inf.
+ *         Inputs are bf16 bit patterns; every product of two bf16 values is
+ *         exact in double, and the double sum is accumulated in h-major,
+ *         d-minor order.  A[b,t,p] = sum_h sum_d |q*c| is returned beside S
+ *         as the scale of the score error bound.
+ * select  "Iterate Topk" (opening description): given per-segment scores,
+ *         return the top-K indices.  Order: descending score; equal scores go
+ *         to the lower index (IEEE equality, so -0 ties with +0: "Round 18
+ *         Track C", section 2, tests signed-zero and adversarial ties).  A page
+ *         is selectable iff p < len and its score is neither -inf nor NaN.
+ *         K' = min(K, #selectable) entries are written, then the slots
+ *         K'..K-1 get index -1 and value -inf.
+ *         The selection is a full sort (C library qsort) of the selectable
+ *         entries under the total order (value desc, index asc); because the
+ *         order is total, the result equals a stable sort by value.
+ *
+ * Error behaviour: every entry point returns 0 on success and -1 when an
+ * argument breaks the contract (negative sizes, len outside [0, N]).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_API __attribute__((visibility("default")))
+
+/* bf16 bit pattern -> double, exactly: the bf16 value is the fp32 value whose
+ * high 16 bits are the pattern and whose low 16 bits are zero. */
+static double bf16_bits_to_double(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* One score and its error-bound scale, by the definition. */
+static void score_one(const uint16_t* q_bt, const uint16_t* c_bp, int Q, int D,
+                      double* s_out, double* a_out)
+{
+    double s = 0.0, a = 0.0;
+    for (int h = 0; h < Q; ++h) {
+        for (int d = 0; d < D; ++d) {
+            double prod = bf16_bits_to_double(q_bt[(int64_t)h * D + d]) *
+                          bf16_bits_to_double(c_bp[d]);
+            s += prod;
+            a += fabs(prod);
+        }
+    }
+    *s_out = s;
+    *a_out = a;
+}
+
+/*
+ * Scores of every (b, t, p).
+ *   q        bf16 bits [B][T][Q][D]
+ *   c        bf16 bits, request b's page p at c + b*ldc_b + p*D  (p < N)
+ *   lengths  [B] valid page counts in [0, N], or NULL for "all N valid"
+ *   S, A     double [B][T][N]; padded entries get S = -inf, A = 0
+ */
+ORACLE_API int oracle_scores(const uint16_t* q, const uint16_t* c,
+                             const int32_t* lengths, int B, int T, int Q, int D,
+                             int N, int64_t ldc_b, double* S, double* A)
+{
+    if (B < 0 || T < 0 || Q <= 0 || D <= 0 || N < 0 || ldc_b < (int64_t)N * D)
+        return -1;
+    for (int b = 0; b < B; ++b) {
+        int len = lengths ? lengths[b] : N;
+        if (len < 0 || len > N) return -1;
+        for (int t = 0; t < T; ++t) {
+            const uint16_t* q_bt = q + ((int64_t)b * T + t) * Q * D;
+            double* s_row = S + ((int64_t)b * T + t) * N;
+            double* a_row = A + ((int64_t)b * T + t) * N;
+            for (int p = 0; p < N; ++p) {
+                if (p >= len) {
+                    s_row[p] = -INFINITY;
+                    a_row[p] = 0.0;
+                    continue;
+                }
+                score_one(q_bt, c + (int64_t)b * ldc_b + (int64_t)p * D, Q, D,
+                          &s_row[p], &a_row[p]);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Scores at n listed (b, t, p) triples, for spot checks at full size. */
+ORACLE_API int oracle_scores_at(const uint16_t* q, const uint16_t* c, int B,
+                                int T, int Q, int D, int N, int64_t ldc_b,
+                                int64_t n, const int32_t* bb, const int32_t* tt,
+                                const int32_t* pp, double* S, double* A)
+{
+    if (Q <= 0 || D <= 0 || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        if (bb[i] < 0 || bb[i] >= B || tt[i] < 0 || tt[i] >= T || pp[i] < 0 ||
+            pp[i] >= N)
+            return -1;
+        score_one(q + ((int64_t)bb[i] * T + tt[i]) * Q * D,
+                  c + (int64_t)bb[i] * ldc_b + (int64_t)pp[i] * D, Q, D, &S[i],
+                  &A[i]);
+    }
+    return 0;
+}
+
+typedef struct {
+    double v;
+    int32_t i;
+} entry;
+
+/* Total order: larger value first; equal values (including -0 == +0) by
+ * ascending index. */
+static int entry_cmp(const void* pa, const void* pb)
+{
+    const entry* a = (const entry*)pa;
+    const entry* b = (const entry*)pb;
+    if (a->v > b->v) return -1;
+    if (a->v < b->v) return 1;
+    return (a->i > b->i) - (a->i < b->i);
+}
+
+/* Core select over a row already widened to double (exact for fp32 input). */
+static int topk_core(const double* row, int len, int K, int32_t* idx_out,
+                     double* val_out)
+{
+    if (len < 0 || K < 0) return -1;
+    entry* e = (entry*)malloc(sizeof(entry) * (size_t)(len > 0 ? len : 1));
+    if (!e) return -1;
+    int n = 0;
+    for (int p = 0; p < len; ++p) {
+        double v = row[p];
+        if (isnan(v) || v == -INFINITY) continue;
+        e[n].v = v;
+        e[n].i = p;
+        ++n;
+    }
+    qsort(e, (size_t)n, sizeof(entry), entry_cmp);
+    int kk = n < K ? n : K;
+    for (int k = 0; k < K; ++k) {
+        idx_out[k] = k < kk ? e[k].i : -1;
+        val_out[k] = k < kk ? e[k].v : -INFINITY;
+    }
+    free(e);
+    return kk;
+}
+
+/* Top-K of one double row; returns K' (the number of real entries) or -1. */
+ORACLE_API int oracle_topk_f64(const double* row, int len, int K,
+                               int32_t* idx_out, double* val_out)
+{
+    return topk_core(row, len, K, idx_out, val_out);
+}
+
+/* Top-K of one fp32 row.  Widening fp32 to double is exact, so every
+ * comparison decides exactly as the same comparison in fp32 would. */
+ORACLE_API int oracle_topk_f32(const float* row, int len, int K,
+                               int32_t* idx_out, float* val_out)
+{
+    if (len < 0 || K < 0) return -1;
+    double* w = (double*)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+    double* v = (double*)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    if (!w || !v) {
+        free(w);
+        free(v);
+        return -1;
+    }
+    for (int p = 0; p < len; ++p) w[p] = (double)row[p];
+    int kk = topk_core(w, len, K, idx_out, v);
+    /* The value written is the row's own fp32 entry (bit-exact, -0 kept). */
+    for (int k = 0; k < K; ++k) val_out[k] = idx_out[k] >= 0 ? row[idx_out[k]] : -INFINITY;
+    free(w);
+    free(v);
+    return kk;
+}
+
+/* Row-batched fp32 select: rows of stride lds, lengths per row (NULL => N). */
+ORACLE_API int oracle_topk_rows_f32(const float* scores, const int32_t* lengths,
+                                    int rows, int N, int64_t lds, int K,
+                                    int32_t* idx_out, float* val_out)
+{
+    if (rows < 0 || N < 0 || K < 0 || lds < N) return -1;
+    for (int r = 0; r < rows; ++r) {
+        int len = lengths ? lengths[r] : N;
+        if (len < 0 || len > N) return -1;
+        if (oracle_topk_f32(scores + (int64_t)r * lds, len, K,
+                            idx_out + (int64_t)r * K, val_out + (int64_t)r * K) < 0)
+            return -1;
+    }
+    return 0;
+}
+
+/* Row-batched double select (the oracle's own scores). */
+ORACLE_API int oracle_topk_rows_f64(const double* scores, const int32_t* lengths,
+                                    int rows, int N, int64_t lds, int K,
+                                    int32_t* idx_out, double* val_out)
+{
+    if (rows < 0 || N < 0 || K < 0 || lds < N) return -1;
+    for (int r = 0; r < rows; ++r) {
+        int len = lengths ? lengths[r] : N;
+        if (len < 0 || len > N) return -1;
+        if (topk_core(scores + (int64_t)r * lds, len, K, idx_out + (int64_t)r * K,
+                      val_out + (int64_t)r * K) < 0)
+            return -1;
+    }
+    return 0;
+}
