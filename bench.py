@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of the page indexer's hot path on B200.
+
+One step = one ``score_topk_fused`` call over a whole batch of the ragged
+decode workload: B=32 requests, Q=4 query heads, D=128, pages per request
+uniform on 1024..65536 inside a padded N=65536, K=256 (seed 103; rank r of a
+multi-GPU run draws its own batch from seed 103 + 1000 r).  Every valid page is
+scored against its request's query heads and the top-K page indices of each
+request are written.  The metric is valid pages scored+selected per second
+(whole job) and the HBM bandwidth that implies.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch under torch.distributed.run: requests are sharded across ranks
+(each rank owns its batch; no collective on the data path), timing is the max
+over ranks.  ``--impl reference`` times the CPU oracle (single-threaded C) on
+a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "pages scored+selected/sec and HBM GB/s vs 8 TB/s at B=32,N=65536,K=256"
+UNIT = "pages/s"
+WORKLOAD = "ragged_decode"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes per valid page of the fused decode kernel, from the ncu capture
+# summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum per
+# launch / pages per launch); None until a capture of the current kernel exists.
+NCU_TRAFFIC_BYTES_PER_PAGE = None
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def workload_inputs(rank):
+    from page_scoring_top_b200 import synth
+    spec = dict(synth.WORKLOADS[WORKLOAD])
+    seed = spec["seed"] + 1000 * rank
+    return synth.workload(WORKLOAD, seed=seed), spec, seed
+
+
+def algorithmic_bytes(lengths, B, T, Q, D, K, with_values):
+    pages = int(np.sum(lengths))
+    b = pages * D * 2 + B * T * Q * D * 2 + B * 4 + B * T * K * 4
+    if with_values:
+        b += B * T * K * 4
+    return pages, b
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[4:8]):
+                if flag.lower() in ("active", "1"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(smax)) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_rate(d, K, seconds, max_requests=None):
+    """Single-threaded oracle (scores in double + full sort per request) on a
+    bounded sample of the workload: whole requests in order, repeated until
+    ``seconds`` elapse (at least one request).  Returns (pages/s, description)."""
+    import oracle
+    q, c, lengths = d["q"], d["c"], d["lengths"]
+    B = q.shape[0]
+    pages = 0
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        b = done % B
+        n = int(lengths[b])
+        S, _ = oracle.scores(q[b:b + 1], c[b:b + 1, :max(n, 1)], np.array([n], np.int32))
+        oracle.topk_rows(S[0], K, None)
+        pages += n
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or (max_requests and done >= max_requests):
+            break
+    return pages / el, "%d requests of the workload in order (%d pages), %.1f s, 1 thread" % (
+        done, pages, el)
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    d, spec, seed = workload_inputs(0)
+    K = spec["K"]
+    import oracle
+    # Calibrate: one request's oracle time, then size each step's sample so the
+    # whole --warmup + --steps run takes about two minutes.
+    t0 = time.perf_counter()
+    n0 = int(d["lengths"][0])
+    S, _ = oracle.scores(d["q"][:1], d["c"][:1, :n0], d["lengths"][:1])
+    oracle.topk_rows(S[0], K, None)
+    per_page = (time.perf_counter() - t0) / n0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    sample_pages = int(max(1024, min(n0, budget / per_page)))
+    total_pages = 0
+    t_total = 0.0
+    for step in range(args.warmup + args.steps):
+        b = step % d["q"].shape[0]
+        n = int(min(sample_pages, d["lengths"][b]))
+        t0 = time.perf_counter()
+        S, _ = oracle.scores(d["q"][b:b + 1], d["c"][b:b + 1, :n], np.array([n], np.int32))
+        oracle.topk_rows(S[0], K, None)
+        el = time.perf_counter() - t0
+        if step >= args.warmup:
+            total_pages += n
+            t_total += el
+    value = total_pages / t_total
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "B": 32, "T": 1, "Q": 4, "D": 128, "N": 65536, "K": K,
+                   "seed": seed, "len_dist": "uniform 1024..65536"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "per step: the first %d valid pages of one request "
+                                   "(requests in turn), scores in double + full sort" %
+                                   sample_pages},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        print("warning: --gpus %d but WORLD_SIZE %d" % (args.gpus, world), file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    from page_scoring_top_b200 import binding
+
+    d, spec, seed = workload_inputs(rank)
+    B, T, Q, D = d["q"].shape
+    N = d["c"].shape[1]
+    K = spec["K"]
+    pages, nbytes = algorithmic_bytes(d["lengths"], B, T, Q, D, K, with_values=False)
+
+    q = torch.from_numpy(d["q"].view(np.int16)).to(dev)
+    c = torch.from_numpy(d["c"].view(np.int16)).to(dev)
+    ln = torch.from_numpy(d["lengths"]).to(dev)
+    idx = torch.empty((B * T, K), dtype=torch.int32, device=dev)
+    ctx = binding.Context(local, max_rows=B * T, max_n=N, max_k=K)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.score_topk_fused(ctx, q, c, ln, K, idx, None, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc, bits = binding.idx_get_status(ctx)
+    if rc != 0:
+        raise RuntimeError("device status %d after warm-up" % bits)
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
+                           os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.15)  # let the sampler take its first reading
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    pages_t = torch.tensor([float(pages)], dtype=torch.float64, device=dev)
+    if pg is not None:
+        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
+        pg.all_reduce(pages_t, op=pg.ReduceOp.SUM)
+    ms_max = float(ms_t.item())
+    ms_per_step = ms_max / args.steps
+    total_pages = float(pages_t.item())
+    value = total_pages * args.steps / (ms_max * 1e-3)
+    rc, bits = binding.idx_get_status(ctx)
+    if rc != 0:
+        raise RuntimeError("device status %d after the timed region" % bits)
+
+    # Roofline of the dominant (only) kernel: the fused decode kernel, one
+    # launch per step on `stream`, timed by the events above.
+    launch_s = (ms / args.steps) * 1e-3
+    achieved = nbytes / launch_s / 1e9
+    peak, peak_src = measured_peak()
+    traffic = None if NCU_TRAFFIC_BYTES_PER_PAGE is None else NCU_TRAFFIC_BYTES_PER_PAGE * pages
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(binding, ctx, d, K, dev, stream, args.e2e_steps, barrier, pg)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, sample = cpu_oracle_rate(d, K, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "T": T, "Q": Q, "D": D, "N": N, "K": K,
+                       "len_dist": "uniform 1024..65536", "seed": seed,
+                       "pages_per_step_per_gpu": pages, "bytes_per_step_per_gpu": nbytes,
+                       "parallelism": "dp%d (requests sharded, no data-path collective)" % world,
+                       "l2": "inputs larger than L2 (%.1f MB of centroids per step vs 126 MB); "
+                             "no flush" % (pages * D * 2 / 1e6)},
+            "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                         "kernel": "decode_kernel<16,1,fused>"},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+def measure_e2e(binding, ctx, d, K, dev, stream, steps, barrier, pg):
+    """The same step through the public call with host buffers: pinned H2D of
+    q, lengths and each request's valid centroid pages, the fused call, and a
+    D2H read of the indices, all inside the timed region."""
+    import torch
+    B, T, Q, D = d["q"].shape
+    N = d["c"].shape[1]
+    q_h = torch.from_numpy(d["q"].view(np.int16)).pin_memory()
+    c_h = torch.from_numpy(d["c"].view(np.int16)).pin_memory()
+    ln_h = torch.from_numpy(d["lengths"]).pin_memory()
+    idx_h = torch.empty((B * T, K), dtype=torch.int32).pin_memory()
+    q = torch.empty_like(q_h, device=dev)
+    c = torch.empty_like(c_h, device=dev)
+    ln = torch.empty_like(ln_h, device=dev)
+    idx = torch.empty((B * T, K), dtype=torch.int32, device=dev)
+    lengths = [int(x) for x in d["lengths"]]
+    h2d = q_h.numel() * 2 + ln_h.numel() * 4 + sum(lengths) * D * 2
+    d2h = idx_h.numel() * 4
+
+    def step():
+        q.copy_(q_h, non_blocking=True)
+        ln.copy_(ln_h, non_blocking=True)
+        for b, n in enumerate(lengths):
+            if n:
+                c[b, :n].copy_(c_h[b, :n], non_blocking=True)
+        binding.score_topk_fused(ctx, q, c, ln, K, idx, None, stream=stream)
+        idx_h.copy_(idx, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = e0.elapsed_time(e1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    pages_t = torch.tensor([float(sum(lengths))], dtype=torch.float64, device=dev)
+    if pg is not None:
+        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
+        pg.all_reduce(pages_t, op=pg.ReduceOp.SUM)
+    value = float(pages_t.item()) * steps / (float(ms_t.item()) * 1e-3)
+    return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps, "ms_per_step": float(ms_t.item()) / steps}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

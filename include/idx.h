@@ -1,0 +1,139 @@
+/*
+ * idx.h -- C ABI of the B200 page indexer (libidx.so).
+ *
+ * The indexer of a block-sparse attention layer scores every candidate KV page
+ * of a request against that request's query heads and keeps the top-K pages
+ * for the sparse attention that follows:
+ *
+ *     s[b,t,p] = sum_{h<Q} sum_{d<D} q[b,t,h,d] * c[b,p,d]        (p < len[b])
+ *     s[b,t,p] = -inf                                               (p >= len[b])
+ *     idx[b,t,:] = the K pages of largest s[b,t,:], by descending score,
+ *                  equal scores to the lower page index.
+ *
+ * Sources: "Iterate Centroids Score" (opening description: score a batch of Q
+ * query rows against a table of block centroids; submission contract
+ * centroid_score(q, centroids, ctx, out)), "Iterate Topk" (opening description:
+ * top-K indices of per-segment scores), "Round 18 Track C: qsa_topk2 ... +
+ * qsa_score ..." (section 1: qsa_score's reduction over heads and dims,
+ * qsa_topk2's radix select over order keys; section 2: ties and signed zero),
+ * "Round 15 Track C Audit" (section 1 Target 1 item 3: a 16-token tile scored
+ * by one matrix product, the dead tail masked).
+ *
+ * Conventions for every call
+ * --------------------------
+ * - Tensors are caller-owned DEVICE memory on the context's device, row-major
+ *   and contiguous unless a stride is given.  bf16 values are passed as their
+ *   uint16_t bit patterns.  Outputs are fully written by the call.
+ * - q       bf16 [B][T][Q][D]                  (T query tokens per request)
+ *   c       bf16, page p of request b at c + b*ldc_b + p*D, p < N
+ *   lengths int32 [B] valid page counts in [0, N], or NULL for "all N valid"
+ *   scores  fp32 [B][T][N]
+ *   idx_out int32 [B*T][K], val_out fp32 [B*T][K] (val_out may be NULL)
+ * - Output rows hold K' = min(K, #selectable pages) entries in order; slots
+ *   K'..K-1 get index -1 and value -inf.  A page is selectable when p < len and
+ *   its score is neither -inf nor NaN; -0 and +0 tie.  val_out[k] is bit-equal
+ *   to the score of page idx_out[k].
+ * - Calls are asynchronous on `stream` (NULL = legacy default stream), never
+ *   allocate and never synchronise the host.  One context must not be used on
+ *   two streams at once: its workspace is shared by its calls.
+ * - Alignment: q, c, scores: 16 bytes; ldc_b*2 bytes a multiple of 16;
+ *   D a multiple of 8 and at most 256.
+ * - Return value: IDX_OK or a negative idx_status.  Argument errors are found
+ *   on the host before anything is launched.  Length VALUES live on the device
+ *   and are not read by the host: a length outside [0, N] is clamped into it on
+ *   the device and reported later by idx_get_status.
+ */
+#ifndef IDX_H_
+#define IDX_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define IDX_API __attribute__((visibility("default")))
+#else
+#define IDX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct idx_ctx idx_ctx;        /* opaque: device, limits, workspace */
+typedef struct CUstream_st* idx_stream; /* the same type as cudaStream_t */
+
+typedef enum {
+  IDX_OK = 0,
+  IDX_EINVAL = -1,        /* null pointer, non-positive size, bad alignment/stride */
+  IDX_EUNSUPPORTED = -2,  /* shape outside what the kernels handle (D, K limits) */
+  IDX_ENOWORKSPACE = -3,  /* rows, N or K beyond the limits given to idx_init */
+  IDX_ECUDA = -4,         /* a CUDA runtime call or kernel launch failed */
+  IDX_EDEVICE = -5        /* device-side status raised (see idx_get_status) */
+} idx_status;
+
+/* Largest K any call accepts. */
+#define IDX_MAX_K 2048
+
+/*
+ * Create a context on `device`.  max_rows bounds B*T, max_n bounds N and max_k
+ * bounds K of every later call; the workspace for those limits is allocated
+ * here, once (the only allocation the library makes), and zeroed.
+ * The two-stage shape (set up once, then cheap repeated calls) follows the
+ * init()/compute() runtime of "Export Cake KMeans plan-runtime suite".
+ * On success *out owns the context; release it with idx_destroy.
+ */
+IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max_k);
+
+/* Free the context and its workspace (synchronises the device first).  NULL is a no-op. */
+IDX_API int idx_destroy(idx_ctx* ctx);
+
+/*
+ * Scores only: scores[b][t][p] for every p < N (-inf for p >= len[b]).
+ * B*T <= max_rows, N <= max_n.  Decode shapes (T*Q small) run on CUDA cores
+ * with the query heads pre-summed in fp32; prefill chunks (T*Q == 128,
+ * D == 128) run a tcgen05 tensor-core product with fp32 accumulation in TMEM.
+ * The fp32 result is within 1e-5 * sum_h sum_d |q_hd * c_pd| of the exact score.
+ */
+IDX_API int centroid_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths,
+                   int B, int T, int Q, int D, int N, int64_t ldc_b, float* scores,
+                   idx_stream stream);
+
+/*
+ * Top-K of fp32 score rows: row r is scores + r*lds, its first len[r] entries
+ * (lengths NULL => N) compete.  rows <= max_rows, N <= max_n, lds >= N,
+ * 1 <= K <= max_k.  Indices are positions within the row.
+ * Exact: the result equals a full sort of the row by (value desc, index asc).
+ */
+IDX_API int topk_select(idx_ctx* ctx, const float* scores, const int32_t* lengths, int rows, int N,
+                int64_t lds, int K, int32_t* idx_out, float* val_out, idx_stream stream);
+
+/*
+ * Score and select in one call: idx_out[b*T+t] = top-K pages of s[b,t,:].
+ * For decode shapes the score row never goes to global memory: each CTA keeps
+ * the scores of its page range in shared memory, selects that range's top-K
+ * candidates there, and the last CTA to finish a row merges the candidates.
+ * Scores are bit-identical to centroid_score's for the same inputs, so the
+ * indices equal topk_select applied to centroid_score's output.
+ */
+IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths,
+                     int B, int T, int Q, int D, int N, int64_t ldc_b, int K, int32_t* idx_out,
+                     float* val_out, idx_stream stream);
+
+/*
+ * Device-side status of the context: waits for `stream`, reads and clears the
+ * status word.  Returns IDX_OK, or IDX_EDEVICE with *bits (if non-NULL) set to
+ * the raised bits: 1 = a length outside [0, N] was clamped, 2 = a bounded wait
+ * inside a kernel expired (that call's output is not valid).  Synchronises.
+ */
+IDX_API int idx_get_status(idx_ctx* ctx, idx_stream stream, int* bits);
+
+/* Static text for a status code. */
+IDX_API const char* idx_strerror(int code);
+
+/* Number of SMs the context sizes its persistent grids for (0 if ctx is NULL). */
+IDX_API int idx_num_sms(const idx_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IDX_H_ */

@@ -1,0 +1,176 @@
+"""Thin Python binding of libidx.so (the C ABI in include/idx.h).
+
+Argument marshalling only: every step of the indexer runs in the CUDA
+library.  The functions keep the C names; tensors are torch CUDA tensors (bf16
+inputs may be given as bfloat16, int16 or uint16 tensors), and the stream
+defaults to torch's current stream on the tensor's device.
+
+If libidx.so is missing the first call raises ``RuntimeError``: there is no
+fallback of any kind.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libidx.so")
+
+IDX_OK, IDX_EINVAL, IDX_EUNSUPPORTED, IDX_ENOWORKSPACE, IDX_ECUDA, IDX_EDEVICE = 0, -1, -2, -3, -4, -5
+IDX_MAX_K = 2048
+
+# Every symbol include/idx.h declares, with its ctypes signature.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_L = ctypes.c_int64
+SIGNATURES = {
+    "idx_init": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I]),
+    "idx_destroy": (_I, [_P]),
+    "centroid_score": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _P, _P]),
+    "topk_select": (_I, [_P, _P, _P, _I, _I, _L, _I, _P, _P, _P]),
+    "score_topk_fused": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _I, _P, _P, _P]),
+    "idx_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
+    "idx_strerror": (ctypes.c_char_p, [_I]),
+    "idx_num_sms": (_I, [_P]),
+}
+
+_lib = None
+
+
+class IdxError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (what, strerror(code), code))
+
+
+def lib():
+    """The loaded CDLL with argtypes set (raises if libidx.so was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libidx.so not found at %s: build it with "
+                               "`python -m page_scoring_top_b200.build`" % LIB_PATH)
+        dll = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(dll, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = dll
+    return _lib
+
+
+def strerror(code):
+    return lib().idx_strerror(int(code)).decode()
+
+
+def _check(rc, what):
+    if rc != IDX_OK:
+        raise IdxError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+class Context:
+    """An idx_ctx: device, limits and the workspace allocated once by idx_init."""
+
+    def __init__(self, device=0, max_rows=1, max_n=1, max_k=1):
+        if isinstance(device, torch.device):
+            device = device.index if device.index is not None else torch.cuda.current_device()
+        self.device = int(device)
+        self.max_rows, self.max_n, self.max_k = int(max_rows), int(max_n), int(max_k)
+        handle = ctypes.c_void_p()
+        _check(lib().idx_init(ctypes.byref(handle), self.device, self.max_rows, self.max_n,
+                              self.max_k), "idx_init")
+        self.handle = handle
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            _check(lib().idx_destroy(self.handle), "idx_destroy")
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    @property
+    def num_sms(self):
+        return lib().idx_num_sms(self.handle)
+
+
+def idx_init(device, max_rows, max_n, max_k):
+    return Context(device, max_rows, max_n, max_k)
+
+
+def idx_destroy(ctx):
+    ctx.close()
+
+
+def _score_shapes(q, c):
+    if q.dim() != 4 or c.dim() != 3:
+        raise ValueError("q must be [B][T][Q][D] and c [B][N][D]")
+    B, T, Q, D = q.shape
+    Bc, N, Dc = c.shape
+    if Bc != B or Dc != D:
+        raise ValueError("q and c disagree on B or D")
+    if not q.is_contiguous() or c.stride(2) != 1 or c.stride(1) != D:
+        raise ValueError("q must be contiguous and c's pages contiguous rows of D")
+    return B, T, Q, D, N, c.stride(0)
+
+
+def centroid_score(ctx, q, c, lengths, scores, stream=None):
+    """scores[b][t][p] (fp32 [B][T][N]) = sum_h q[b,t,h,:] . c[b,p,:]; -inf past lengths."""
+    B, T, Q, D, N, ldc = _score_shapes(q, c)
+    if tuple(scores.shape) != (B, T, N) or scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous fp32 [B][T][N]")
+    _check(lib().centroid_score(ctx.handle, _ptr(q), _ptr(c), _ptr(lengths), B, T, Q, D, N, ldc,
+                                _ptr(scores), _stream(stream, q.device)), "centroid_score")
+    return scores
+
+
+def topk_select(ctx, scores, lengths, K, idx_out, val_out=None, stream=None):
+    """Top-K of each row of a 2-D fp32 tensor (row stride = scores.stride(0))."""
+    if scores.dim() != 2 or scores.stride(1) != 1:
+        raise ValueError("scores must be 2-D with unit column stride")
+    rows, N = scores.shape
+    _check(lib().topk_select(ctx.handle, _ptr(scores), _ptr(lengths), rows, N, scores.stride(0), K,
+                             _ptr(idx_out), _ptr(val_out), _stream(stream, scores.device)),
+           "topk_select")
+    return idx_out, val_out
+
+
+def score_topk_fused(ctx, q, c, lengths, K, idx_out, val_out=None, stream=None):
+    """idx_out[b*T+t] = top-K pages of request b for token t (int32 [B*T][K])."""
+    B, T, Q, D, N, ldc = _score_shapes(q, c)
+    _check(lib().score_topk_fused(ctx.handle, _ptr(q), _ptr(c), _ptr(lengths), B, T, Q, D, N, ldc,
+                                  K, _ptr(idx_out), _ptr(val_out), _stream(stream, q.device)),
+           "score_topk_fused")
+    return idx_out, val_out
+
+
+def idx_get_status(ctx, stream=None):
+    """(status code, raised bits) of the context; synchronises the stream."""
+    bits = ctypes.c_int(0)
+    rc = lib().idx_get_status(ctx.handle, _stream(stream, torch.device("cuda", ctx.device)),
+                              ctypes.byref(bits))
+    return rc, bits.value

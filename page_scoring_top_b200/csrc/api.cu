@@ -1,0 +1,324 @@
+// api.cu -- the C ABI of libidx.so: argument checks, workspace, dispatch.
+//
+// The context follows the two-stage runtime shape of "Export Cake KMeans
+// plan-runtime suite" (summary: init() once, then compute() many times): all
+// device memory the kernels need is sized from the caller's limits and
+// allocated in idx_init; every later call only validates, picks a kernel and
+// launches it on the caller's stream.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "idx.h"
+#include "kernels.h"
+
+struct idx_ctx {
+  int device;
+  int max_rows, max_n, max_k;
+  int num_sms;
+  void* ws;  // one allocation holding everything below
+  size_t ws_bytes;
+  uint32_t* cand_bits;
+  int32_t* cand_idx;
+  int32_t* cand_cnt;
+  int64_t cand_slots;
+  int32_t* arrive;
+  int* status;
+  float* scratch;  // fp32 scores for the score-then-select route
+  int64_t scratch_elems;
+};
+
+namespace {
+
+// Runs the body with ctx->device current, restoring the caller's device.
+class DeviceGuard {
+ public:
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev_) != cudaSuccess) prev_ = -1;
+    if (prev_ != dev) ok_ = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev_ >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev_) cudaSetDevice(prev_);
+  }
+  bool ok() const { return ok_; }
+
+ private:
+  int prev_ = -1;
+  bool ok_ = true;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int check_score_args(const idx_ctx* ctx, const uint16_t* q, const uint16_t* c, int B, int T,
+                     int Q, int D, int N, int64_t ldc_b) {
+  if (!ctx || !q || !c) return IDX_EINVAL;
+  if (B <= 0 || T <= 0 || Q <= 0 || D <= 0 || N <= 0) return IDX_EINVAL;
+  if (!aligned16(q) || !aligned16(c)) return IDX_EINVAL;
+  if (ldc_b < (int64_t)N * D || (ldc_b % 8) != 0) return IDX_EINVAL;
+  if ((D % 8) != 0 || D > 256) return IDX_EUNSUPPORTED;
+  if ((int64_t)B * T > ctx->max_rows || N > ctx->max_n) return IDX_ENOWORKSPACE;
+  if ((int64_t)B * N > INT32_MAX) return IDX_EUNSUPPORTED;
+  return IDX_OK;
+}
+
+int check_k(const idx_ctx* ctx, int K) {
+  if (K <= 0) return IDX_EINVAL;
+  if (K > IDX_MAX_K) return IDX_EUNSUPPORTED;
+  if (K > ctx->max_k) return IDX_ENOWORKSPACE;
+  return IDX_OK;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? IDX_OK : IDX_ECUDA; }
+
+int run_topk(idx_ctx* ctx, const float* scores, const int32_t* lengths, int len_div, int rows,
+             int N, int64_t lds, int K, int32_t* idx_out, float* val_out, cudaStream_t stream) {
+  idx::TopkArgs a{};
+  a.scores = scores;
+  a.lengths = lengths;
+  a.len_div = len_div;
+  a.rows = rows;
+  a.N = N;
+  a.lds = lds;
+  a.K = K;
+  a.chunk = idx::topk_plan_chunk(rows, N, K, ctx->num_sms);
+  a.max_chunks = (int)ceil_div(N, a.chunk);
+  if ((int64_t)rows * a.max_chunks > ctx->cand_slots) return IDX_ENOWORKSPACE;
+  a.idx_out = idx_out;
+  a.val_out = val_out;
+  a.cand_bits = ctx->cand_bits;
+  a.cand_idx = ctx->cand_idx;
+  a.cand_cnt = ctx->cand_cnt;
+  a.slot_stride = ctx->max_k;
+  a.arrive = ctx->arrive;
+  a.status = ctx->status;
+  return status_of(idx::launch_topk(a, stream));
+}
+
+int run_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths, int B,
+              int T, int Q, int D, int N, int64_t ldc_b, float* scores, cudaStream_t stream) {
+  if (idx::prefill_supported(T, Q, D, ldc_b)) {
+    idx::PrefillArgs p{};
+    p.q = q;
+    p.c = c;
+    p.lengths = lengths;
+    p.B = B;
+    p.T = T;
+    p.Q = Q;
+    p.D = D;
+    p.N = N;
+    p.ldc_b = ldc_b;
+    p.scores = scores;
+    p.status = ctx->status;
+    return status_of(idx::launch_prefill(p, ctx->num_sms, stream));
+  }
+  for (int b0 = 0; b0 < B; b0 += idx::kDecodeMaxB) {
+    const int nb = std::min(idx::kDecodeMaxB, B - b0);
+    idx::DecodeArgs a{};
+    a.q = q + (int64_t)b0 * T * Q * D;
+    a.c = c + (int64_t)b0 * ldc_b;
+    a.lengths = lengths ? lengths + b0 : nullptr;
+    a.B = nb;
+    a.T = T;
+    a.Q = Q;
+    a.D = D;
+    a.N = N;
+    a.ldc_b = ldc_b;
+    a.scores = scores + (int64_t)b0 * T * N;
+    a.status = ctx->status;
+    const int rc = status_of(idx::launch_decode(a, false, ctx->num_sms, stream));
+    if (rc != IDX_OK) return rc;
+  }
+  return IDX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max_k) {
+  if (!out) return IDX_EINVAL;
+  *out = nullptr;
+  if (max_rows <= 0 || max_n <= 0 || max_k <= 0) return IDX_EINVAL;
+  if (max_k > IDX_MAX_K) return IDX_EUNSUPPORTED;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return IDX_ECUDA;
+  DeviceGuard guard(device);
+  if (!guard.ok()) return IDX_ECUDA;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return IDX_ECUDA;
+
+  idx_ctx* ctx = new idx_ctx();
+  ctx->device = device;
+  ctx->max_rows = max_rows;
+  ctx->max_n = max_n;
+  ctx->max_k = max_k;
+  ctx->num_sms = sms;
+  // Candidate slots: the larger of the standalone select's (rows x chunks of
+  // at least 2048 entries) and the fused decode path's (chunks + requests).
+  const int64_t topk_slots = (int64_t)max_rows * ceil_div(max_n, 2048);
+  int64_t fused_slots = 0;
+  for (int t = 1; t <= idx::kDecodeMaxTFused; ++t) {
+    const int64_t b = std::min<int64_t>(max_rows / t, idx::kDecodeMaxB);
+    if (b > 0)
+      fused_slots = std::max(fused_slots,
+                             idx::decode_fused_slots(b, t, max_n, idx::decode_grid(sms)));
+  }
+  ctx->cand_slots = std::max(topk_slots, fused_slots);
+  ctx->scratch_elems = (int64_t)max_rows * max_n;
+  size_t off = 0;
+  auto carve = [&](size_t bytes) {
+    size_t o = off;
+    off += (bytes + 255) & ~(size_t)255;
+    return o;
+  };
+  const size_t o_bits = carve((size_t)ctx->cand_slots * max_k * 4);
+  const size_t o_idx = carve((size_t)ctx->cand_slots * max_k * 4);
+  const size_t o_cnt = carve((size_t)ctx->cand_slots * 4);
+  const size_t o_arr = carve((size_t)max_rows * 4);
+  const size_t o_st = carve(16);
+  const size_t o_scr = carve((size_t)ctx->scratch_elems * 4);
+  ctx->ws_bytes = off;
+  char* base = nullptr;
+  if (cudaMalloc(&base, off) != cudaSuccess) {
+    delete ctx;
+    return IDX_ECUDA;
+  }
+  // Counters and the status word start at zero; kernels return them to zero.
+  if (cudaMemset(base + o_cnt, 0, o_scr - o_cnt) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(base);
+    delete ctx;
+    return IDX_ECUDA;
+  }
+  ctx->ws = base;
+  ctx->cand_bits = reinterpret_cast<uint32_t*>(base + o_bits);
+  ctx->cand_idx = reinterpret_cast<int32_t*>(base + o_idx);
+  ctx->cand_cnt = reinterpret_cast<int32_t*>(base + o_cnt);
+  ctx->arrive = reinterpret_cast<int32_t*>(base + o_arr);
+  ctx->status = reinterpret_cast<int*>(base + o_st);
+  ctx->scratch = reinterpret_cast<float*>(base + o_scr);
+  *out = ctx;
+  return IDX_OK;
+}
+
+IDX_API int idx_destroy(idx_ctx* ctx) {
+  if (!ctx) return IDX_OK;
+  int rc = IDX_OK;
+  {
+    DeviceGuard guard(ctx->device);
+    if (cudaDeviceSynchronize() != cudaSuccess) rc = IDX_ECUDA;
+    if (cudaFree(ctx->ws) != cudaSuccess) rc = IDX_ECUDA;
+  }
+  delete ctx;
+  return rc;
+}
+
+IDX_API int centroid_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                           const int32_t* lengths, int B, int T, int Q, int D, int N,
+                           int64_t ldc_b, float* scores, idx_stream stream) {
+  int rc = check_score_args(ctx, q, c, B, T, Q, D, N, ldc_b);
+  if (rc != IDX_OK) return rc;
+  if (!scores || !aligned16(scores)) return IDX_EINVAL;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  return run_score(ctx, q, c, lengths, B, T, Q, D, N, ldc_b, scores, (cudaStream_t)stream);
+}
+
+IDX_API int topk_select(idx_ctx* ctx, const float* scores, const int32_t* lengths, int rows,
+                        int N, int64_t lds, int K, int32_t* idx_out, float* val_out,
+                        idx_stream stream) {
+  if (!ctx || !scores || !idx_out) return IDX_EINVAL;
+  if (rows <= 0 || N <= 0 || lds < N) return IDX_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(scores) & 3) != 0) return IDX_EINVAL;
+  int rc = check_k(ctx, K);
+  if (rc != IDX_OK) return rc;
+  if (rows > ctx->max_rows || N > ctx->max_n) return IDX_ENOWORKSPACE;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  return run_topk(ctx, scores, lengths, 1, rows, N, lds, K, idx_out, val_out,
+                  (cudaStream_t)stream);
+}
+
+IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                             const int32_t* lengths, int B, int T, int Q, int D, int N,
+                             int64_t ldc_b, int K, int32_t* idx_out, float* val_out,
+                             idx_stream stream) {
+  int rc = check_score_args(ctx, q, c, B, T, Q, D, N, ldc_b);
+  if (rc != IDX_OK) return rc;
+  if (!idx_out) return IDX_EINVAL;
+  rc = check_k(ctx, K);
+  if (rc != IDX_OK) return rc;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (T <= idx::kDecodeMaxTFused && !idx::prefill_supported(T, Q, D, ldc_b)) {
+    for (int b0 = 0; b0 < B; b0 += idx::kDecodeMaxB) {
+      const int nb = std::min(idx::kDecodeMaxB, B - b0);
+      idx::DecodeArgs a{};
+      a.q = q + (int64_t)b0 * T * Q * D;
+      a.c = c + (int64_t)b0 * ldc_b;
+      a.lengths = lengths ? lengths + b0 : nullptr;
+      a.B = nb;
+      a.T = T;
+      a.Q = Q;
+      a.D = D;
+      a.N = N;
+      a.ldc_b = ldc_b;
+      a.K = K;
+      a.idx_out = idx_out + (int64_t)b0 * T * K;
+      a.val_out = val_out ? val_out + (int64_t)b0 * T * K : nullptr;
+      a.cand_bits = ctx->cand_bits;
+      a.cand_idx = ctx->cand_idx;
+      a.cand_cnt = ctx->cand_cnt;
+      a.slot_stride = ctx->max_k;
+      a.arrive = ctx->arrive;
+      a.status = ctx->status;
+      if (idx::decode_fused_slots(nb, T, N, idx::decode_grid(ctx->num_sms)) > ctx->cand_slots)
+        return IDX_ENOWORKSPACE;
+      rc = status_of(idx::launch_decode(a, true, ctx->num_sms, st));
+      if (rc != IDX_OK) return rc;
+    }
+    return IDX_OK;
+  }
+  // Prefill chunks (and token counts beyond the fused CUDA-core path): score
+  // into the context's scratch, then select each (request, token) row.
+  if ((int64_t)B * T * N > ctx->scratch_elems) return IDX_ENOWORKSPACE;
+  rc = run_score(ctx, q, c, lengths, B, T, Q, D, N, ldc_b, ctx->scratch, st);
+  if (rc != IDX_OK) return rc;
+  return run_topk(ctx, ctx->scratch, lengths, T, B * T, N, N, K, idx_out, val_out, st);
+}
+
+IDX_API int idx_get_status(idx_ctx* ctx, idx_stream stream, int* bits) {
+  if (!ctx) return IDX_EINVAL;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  int h = 0;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return IDX_ECUDA;
+  if (cudaMemcpy(&h, ctx->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return IDX_ECUDA;
+  if (cudaMemset(ctx->status, 0, sizeof(int)) != cudaSuccess) return IDX_ECUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return IDX_ECUDA;
+  if (bits) *bits = h;
+  return h ? IDX_EDEVICE : IDX_OK;
+}
+
+IDX_API const char* idx_strerror(int code) {
+  switch (code) {
+    case IDX_OK: return "ok";
+    case IDX_EINVAL: return "invalid argument (null pointer, size, alignment or stride)";
+    case IDX_EUNSUPPORTED: return "unsupported shape (D must be a multiple of 8 up to 256; K up to 2048)";
+    case IDX_ENOWORKSPACE: return "rows, N or K exceed the limits given to idx_init";
+    case IDX_ECUDA: return "CUDA runtime error or kernel launch failure";
+    case IDX_EDEVICE: return "device-side status raised (clamped length or expired wait)";
+    default: return "unknown status";
+  }
+}
+
+IDX_API int idx_num_sms(const idx_ctx* ctx) { return ctx ? ctx->num_sms : 0; }
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// kernels.h -- internal launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace idx {
+
+// ---------------------------------------------------------------- top-K select
+struct TopkArgs {
+  const float* scores;
+  const int32_t* lengths;  // or null (all N); row r uses lengths[r / len_div]
+  int len_div;
+  int rows, N;
+  int64_t lds;
+  int K;
+  int chunk;       // elements per CTA (power of two)
+  int max_chunks;  // candidate slots per row
+  int64_t slot_stride;  // entries per candidate slot (>= K)
+  int32_t* idx_out;
+  float* val_out;  // may be null
+  uint32_t* cand_bits;
+  int32_t* cand_idx;
+  int32_t* cand_cnt;
+  int32_t* arrive;  // per-row arrival counters, zero between calls
+  int* status;
+};
+// Candidate slots the launch needs: rows * max_chunks, each of K entries.
+int topk_plan_chunk(int rows, int N, int K, int num_sms);
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode score / fused select
+struct DecodeArgs {
+  const uint16_t* q;
+  const uint16_t* c;
+  const int32_t* lengths;  // per request, or null
+  int B, T, Q, D, N;
+  int64_t ldc_b;
+  int K;
+  float* scores;    // score mode: [B][T][N]
+  int32_t* idx_out; // fused mode: [B*T][K]
+  float* val_out;   // fused mode, may be null
+  uint32_t* cand_bits;
+  int32_t* cand_idx;
+  int32_t* cand_cnt;
+  int64_t slot_stride;  // entries per candidate slot (>= K)
+  int32_t* arrive;      // per-request arrival counters, zero between calls
+  int* status;
+};
+constexpr int kDecodeMaxB = 1024;       // requests per launch (host splits larger batches)
+constexpr int kDecodeMaxTFused = 4;     // tokens per request on the fused CUDA-core path
+constexpr int kDecodeScoreCap = 16384;  // fused: fp32 scores a CTA keeps on chip
+// Candidate slots a fused launch of B requests x T tokens can use.
+int64_t decode_fused_slots(int64_t B, int64_t T, int64_t N, int grid);
+int decode_grid(int num_sms);
+cudaError_t launch_decode(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream);
+
+// ---------------------------------------------------------------- prefill (tcgen05) score
+struct PrefillArgs {
+  const uint16_t* q;
+  const uint16_t* c;
+  const int32_t* lengths;
+  int B, T, Q, D, N;
+  int64_t ldc_b;
+  float* scores;  // [B][T][N]
+  int* status;
+};
+bool prefill_supported(int T, int Q, int D, int64_t ldc_b);
+cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t stream);
+
+}  // namespace idx
