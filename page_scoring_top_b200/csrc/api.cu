@@ -21,7 +21,7 @@ struct idx_ctx {
   size_t ws_bytes;
   uint32_t* cand_bits;
   int32_t* cand_idx;
-  int32_t* cand_cnt;
+  unsigned long long* row_thr;
   int64_t cand_slots;
   int32_t* arrive;
   int* status;
@@ -91,7 +91,7 @@ int run_topk(idx_ctx* ctx, const float* scores, const int32_t* lengths, int len_
   a.val_out = val_out;
   a.cand_bits = ctx->cand_bits;
   a.cand_idx = ctx->cand_idx;
-  a.cand_cnt = ctx->cand_cnt;
+  a.row_thr = ctx->row_thr;
   a.slot_stride = ctx->max_k;
   a.arrive = ctx->arrive;
   a.status = ctx->status;
@@ -178,7 +178,7 @@ IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max
   };
   const size_t o_bits = carve((size_t)ctx->cand_slots * max_k * 4);
   const size_t o_idx = carve((size_t)ctx->cand_slots * max_k * 4);
-  const size_t o_cnt = carve((size_t)ctx->cand_slots * 4);
+  const size_t o_thr = carve((size_t)max_rows * 8);
   const size_t o_arr = carve((size_t)max_rows * 4);
   const size_t o_st = carve(16);
   const size_t o_scr = carve((size_t)ctx->scratch_elems * 4);
@@ -188,8 +188,9 @@ IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max
     delete ctx;
     return IDX_ECUDA;
   }
-  // Counters and the status word start at zero; kernels return them to zero.
-  if (cudaMemset(base + o_cnt, 0, o_scr - o_cnt) != cudaSuccess ||
+  // Thresholds, counters and the status word start at zero; kernels return
+  // them to zero.
+  if (cudaMemset(base + o_thr, 0, o_scr - o_thr) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(base);
     delete ctx;
@@ -198,7 +199,7 @@ IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max
   ctx->ws = base;
   ctx->cand_bits = reinterpret_cast<uint32_t*>(base + o_bits);
   ctx->cand_idx = reinterpret_cast<int32_t*>(base + o_idx);
-  ctx->cand_cnt = reinterpret_cast<int32_t*>(base + o_cnt);
+  ctx->row_thr = reinterpret_cast<unsigned long long*>(base + o_thr);
   ctx->arrive = reinterpret_cast<int32_t*>(base + o_arr);
   ctx->status = reinterpret_cast<int*>(base + o_st);
   ctx->scratch = reinterpret_cast<float*>(base + o_scr);
@@ -256,7 +257,8 @@ IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
   DeviceGuard guard(ctx->device);
   if (!guard.ok()) return IDX_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  if (T <= idx::kDecodeMaxTFused && !idx::prefill_supported(T, Q, D, ldc_b)) {
+  if (T <= idx::kDecodeMaxTFused && K <= idx::decode_fused_max_k(T) &&
+      !idx::prefill_supported(T, Q, D, ldc_b)) {
     for (int b0 = 0; b0 < B; b0 += idx::kDecodeMaxB) {
       const int nb = std::min(idx::kDecodeMaxB, B - b0);
       idx::DecodeArgs a{};
@@ -274,7 +276,7 @@ IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
       a.val_out = val_out ? val_out + (int64_t)b0 * T * K : nullptr;
       a.cand_bits = ctx->cand_bits;
       a.cand_idx = ctx->cand_idx;
-      a.cand_cnt = ctx->cand_cnt;
+      a.row_thr = ctx->row_thr;
       a.slot_stride = ctx->max_k;
       a.arrive = ctx->arrive;
       a.status = ctx->status;

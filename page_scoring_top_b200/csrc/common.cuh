@@ -16,6 +16,12 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+// Optional timing trace points: IDX_TRACE(i) is empty unless a profiling build
+// defines it (for example to record %globaltimer into a per-CTA buffer).
+#ifndef IDX_TRACE
+#define IDX_TRACE(i)
+#endif
+
 namespace idx {
 
 // ----------------------------------------------------------------- status bits
@@ -87,10 +93,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(2000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -99,7 +105,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // status bit kErrWaitTimeout is raised, *abort is set, and false is returned;
 // once *abort is set every later wait returns at once, so a CTA whose data
 // never arrives still runs to its end through the same barriers.
-constexpr uint32_t kMaxWaitIters = 1u << 20;  // with a 2 us suspend hint: ~2 s
+constexpr uint32_t kMaxWaitIters = 1u << 24;  // each try_wait blocks for a bounded, short time
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort, int* status) {
@@ -123,195 +129,20 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+__device__ __forceinline__ void bulk_g2s_nohint(void* dst, const void* src, uint32_t bytes,
+                                                uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 
-// ----------------------------------------------------------------- block select
-struct SelectScratch {
-  uint32_t hist[2048 + 2048 + 1024];  // passes 1, 2, 3
-  uint32_t wsum[32];
-  uint32_t wsum2[32];
-  uint32_t bcast[4];
-};
-
-// Among bins hist[0..nb) find b with suffix(b+1) < r <= suffix(b), where
-// suffix(x) = sum_{y >= x} hist[y].  Result in sc.bcast[0] (bin) and
-// sc.bcast[1] (suffix(b+1)).  nb must be a multiple of NT.
-template <int NT>
-__device__ __forceinline__ void find_rank_bin(const uint32_t* hist, int nb, uint32_t r,
-                                              SelectScratch& sc) {
-  const int tid = threadIdx.x;
-  const int bpt = nb / NT;
-  const int hi = nb - tid * bpt;  // thread 0 owns the top bins
-  uint32_t s = 0;
-  for (int k = 1; k <= bpt; ++k) s += hist[hi - k];
-  const uint32_t incl = warp_incl_scan(s);
-  const int warp = tid >> 5;
-  if (lane_id() == 31) sc.wsum[warp] = incl;
-  group_sync(NT);
-  uint32_t excl = incl - s;
-  for (int w = 0; w < warp; ++w) excl += sc.wsum[w];
-  if (excl < r && r <= excl + s) {
-    uint32_t cum = excl;
-    for (int k = 1; k <= bpt; ++k) {
-      const uint32_t c = hist[hi - k];
-      if (cum + c >= r) {
-        sc.bcast[0] = (uint32_t)(hi - k);
-        sc.bcast[1] = cum;
-        break;
-      }
-      cum += c;
-    }
-  }
-  group_sync(NT);
-}
-
-// Exact ordered top-K of s_bits[0..n) (fp32 bit patterns in shared memory;
-// position = rank of the page/element index).  Called by the first NT
-// threads of the block, all together.  The winners -- every valid key above
-// the K'-th largest key tau, plus the lowest positions whose key equals tau --
-// go to win_pos[0..K') in ascending position order.  Returns K' =
-// min(K, #valid).  win_pos needs K entries.
-template <int NT>
-__device__ int block_select(const uint32_t* s_bits, int n, int K, int* win_pos,
-                            SelectScratch& sc) {
-  static_assert(NT % 32 == 0 && 1024 % NT == 0, "NT must divide 1024");
-  const int tid = threadIdx.x;
-  uint32_t* h1 = sc.hist;
-  uint32_t* h2 = h1 + 2048;
-  uint32_t* h3 = h2 + 2048;
-  for (int i = tid; i < 2048 + 2048 + 1024; i += NT) sc.hist[i] = 0u;
-  group_sync(NT);
-  for (int i = tid; i < n; i += NT) atomicAdd(&h1[order_key(s_bits[i]) >> 21], 1u);
-  group_sync(NT);
-  const uint32_t valid = (uint32_t)n - h1[0];
-  group_sync(NT);  // everyone has read h1[0] before anyone may reuse the scratch
-  const uint32_t kk = min((uint32_t)K, valid);
-  if (kk == 0) return 0;
-  uint32_t tau = 0, need = 0;  // tau = 0, need = 0: every valid key wins
-  if (kk < valid) {
-    find_rank_bin<NT>(h1, 2048, kk, sc);
-    const uint32_t b1 = sc.bcast[0];
-    uint32_t r = kk - sc.bcast[1];
-    for (int i = tid; i < n; i += NT) {
-      const uint32_t k = order_key(s_bits[i]);
-      if ((k >> 21) == b1) atomicAdd(&h2[(k >> 10) & 2047u], 1u);
-    }
-    group_sync(NT);
-    find_rank_bin<NT>(h2, 2048, r, sc);
-    const uint32_t b2 = sc.bcast[0];
-    r -= sc.bcast[1];
-    const uint32_t pre = (b1 << 11) | b2;
-    for (int i = tid; i < n; i += NT) {
-      const uint32_t k = order_key(s_bits[i]);
-      if ((k >> 10) == pre) atomicAdd(&h3[k & 1023u], 1u);
-    }
-    group_sync(NT);
-    find_rank_bin<NT>(h3, 1024, r, sc);
-    tau = (pre << 10) | sc.bcast[0];
-    need = r - sc.bcast[1];
-  }
-  // Ordered compaction: warp w owns a contiguous span, lanes interleaved.
-  constexpr int NW = NT / 32;
-  const int warp = tid >> 5;
-  const int span = (((n + NW - 1) / NW) + 31) & ~31;
-  const int beg = warp * span;
-  const int end = min(beg + span, n);
-  uint32_t c_gt = 0, c_eq = 0;
-  for (int base = beg; base < end; base += 32) {
-    const int i = base + (int)lane_id();
-    const uint32_t k = (i < end) ? order_key(s_bits[i]) : kKeyInvalid;
-    c_gt += __popc(__ballot_sync(0xFFFFFFFFu, k > tau));
-    c_eq += __popc(__ballot_sync(0xFFFFFFFFu, need > 0 && i < end && k == tau));
-  }
-  if (lane_id() == 0) {
-    sc.wsum[warp] = c_gt;
-    sc.wsum2[warp] = c_eq;
-  }
-  group_sync(NT);
-  uint32_t gt_before = 0, eq_seen = 0;
-  for (int w = 0; w < warp; ++w) {
-    gt_before += sc.wsum[w];
-    eq_seen += sc.wsum2[w];
-  }
-  uint32_t out = gt_before + min(eq_seen, need);
-  const uint32_t lt = lanemask_lt();
-  for (int base = beg; base < end; base += 32) {
-    const int i = base + (int)lane_id();
-    const uint32_t k = (i < end) ? order_key(s_bits[i]) : kKeyInvalid;
-    const bool eq = need > 0 && i < end && k == tau;
-    const uint32_t meq = __ballot_sync(0xFFFFFFFFu, eq);
-    const bool take = (k > tau) || (eq && (eq_seen + __popc(meq & lt) < need));
-    const uint32_t mt = __ballot_sync(0xFFFFFFFFu, take);
-    if (take) win_pos[out + __popc(mt & lt)] = i;
-    out += __popc(mt);
-    eq_seen += __popc(meq);
-  }
-  group_sync(NT);
-  return (int)kk;
-}
-
-// Bitonic sort, descending, of buf[0..P2) (P2 a power of two) by the first
-// NT threads.  Entries are (order key << 32) | ~position, so equal keys come
-// out in ascending position order; padding entries are 0 and sort last.
-template <int NT>
-__device__ void block_sort_desc(uint64_t* buf, int P2) {
-  for (int size = 2; size <= P2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < (P2 >> 1); i += NT) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = (lo & size) == 0;
-        const uint64_t a = buf[lo], b = buf[hi];
-        if ((a < b) == desc) {
-          buf[lo] = b;
-          buf[hi] = a;
-        }
-      }
-      group_sync(NT);
-    }
-  }
-}
-
-__host__ __device__ __forceinline__ int next_pow2(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
-// Sort the K' winners named by win_pos (positions into bits[]) and write the
-// final row: idx_out[k] = gidx[pos] (or base + pos when gidx is null), val_out
-// the exact fp32 bits; slots K'..K-1 get -1 / -inf.  sortbuf holds
-// next_pow2(K) entries.
-template <int NT>
-__device__ void sort_and_write(const uint32_t* bits, const int32_t* gidx, int32_t base,
-                               const int* win_pos, int kk, int K, uint64_t* sortbuf,
-                               int32_t* idx_out, float* val_out) {
-  const int P2 = next_pow2(max(kk, 1));
-  for (int i = threadIdx.x; i < P2; i += NT) {
-    uint64_t e = 0;
-    if (i < kk) {
-      const uint32_t pos = (uint32_t)win_pos[i];
-      e = ((uint64_t)order_key(bits[pos]) << 32) | (uint64_t)(~pos);
-    }
-    sortbuf[i] = e;
-  }
-  group_sync(NT);
-  block_sort_desc<NT>(sortbuf, P2);
-  for (int k = threadIdx.x; k < K; k += NT) {
-    if (k < kk) {
-      const uint32_t pos = ~(uint32_t)(sortbuf[k] & 0xFFFFFFFFull);
-      idx_out[k] = gidx ? gidx[pos] : base + (int32_t)pos;
-      if (val_out) val_out[k] = __uint_as_float(bits[pos]);
-    } else {
-      idx_out[k] = -1;
-      if (val_out) val_out[k] = __uint_as_float(kNegInfBits);
-    }
-  }
-  group_sync(NT);
-}
 
 }  // namespace idx

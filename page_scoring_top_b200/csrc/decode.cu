@@ -17,21 +17,23 @@
 //  * Warp 8 is the producer: one lane streams 32-page stages of the centroid
 //    table into a shared-memory ring with 1-D bulk copies (TMA engine), an
 //    mbarrier pair per slot, L2 evict-first.
-//  * Warps 0..7 consume stages round-robin.  D/8 lanes cover one page's
-//    16-byte chunks (32/(D/8) pages per warp instruction, conflict-free), each
-//    lane keeps its 8 pre-summed query values in registers, and a transposed
-//    butterfly of shuffles leaves lane l holding one page's full score.
-//  * Score mode writes the scores (and -inf padding) to HBM.  Fused mode keeps
-//    the chunk's scores in shared memory; when a row's part of the chunk is
-//    done, the consumer warps select its exact top-K' there, publish the
-//    candidates, and the last CTA to finish the row merges all of the row's
-//    candidates and writes the final indices.  The full score row never
-//    reaches HBM, and the producer keeps prefetching during the select.
+//  * Warps 0..7 consume stages round-robin.  Four lanes share a page (8 pages
+//    per warp instruction); lane c of page-group p reads the page's 16-byte
+//    chunks c, c+4, ... starting at a rotation (p mod chunks-per-lane) that
+//    makes every 128-byte shared-memory wavefront hit 32 distinct banks.  Each
+//    lane keeps its pre-summed query chunks in registers; a two-step butterfly
+//    of shuffles leaves each lane with one page's full score.
+//  * Score mode writes the scores (and -inf padding) to HBM.  Fused mode offers
+//    each score to an exact online top-K filter in shared memory (select.cuh);
+//    at the end of a row's part of the chunk the filter is compacted to K
+//    candidates, published, and the last CTA to finish the row merges all of
+//    the row's candidates and writes the final indices.  The score row never
+//    reaches HBM and the producer keeps prefetching through every compaction.
 // Both modes run the same arithmetic, so fused and score-mode scores are
 // bit-identical.
 #include "common.cuh"
 #include "kernels.h"
-#include "merge.cuh"
+#include "select.cuh"
 
 namespace idx {
 
@@ -40,43 +42,58 @@ constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumers + 32;
 constexpr int kStagePages = 32;
 constexpr int kMaxStages = 32;
-constexpr int kLMin = 128;
+constexpr int kLMin = 256;
 constexpr int kSmemMax = 227 * 1024;
+constexpr int kMaxFusedT = 4;
+constexpr int kProducerLanes = 4;
+constexpr size_t kRingTargetBytes = 128 * 1024;
 
 struct DecodeLayout {
-  size_t ring, score, win, scratch, off, bar, misc, total;
+  size_t ring, fbuf, fstate, scratch, sortv, sortb, off, bar, misc, total;
   int nstage;
+  int cap;  // filter entries per token
 };
 
-__host__ __device__ inline DecodeLayout decode_layout(bool fused, int D) {
+__host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+// Shared-memory layout; identical on host (launch size) and device.
+__host__ __device__ inline DecodeLayout decode_layout(bool fused, int D, int T) {
   DecodeLayout L;
   const size_t stage_bytes = (size_t)kStagePages * D * 2;
-  size_t fixed = 0;
-  fixed += fused ? (size_t)kDecodeScoreCap * 4 : 0;                       // score
-  fixed += fused ? 2048 * 4 : 0;                                          // win_pos
-  fixed += fused ? ((sizeof(SelectScratch) + 15) & ~(size_t)15) : 0;     // scratch / sort
-  fixed += (size_t)(kDecodeMaxB + 1) * 4 + 12;                            // off (+pad)
-  fixed += (size_t)2 * kMaxStages * 8;                                    // barriers
-  fixed += 64;                                                            // misc
-  size_t ring_cap = (size_t)kSmemMax - fixed;
-  int ns = (int)(ring_cap / stage_bytes);
-  if (ns > kMaxStages) ns = kMaxStages;
-  L.nstage = ns;
+  int tp = 1;
+  while (tp < T) tp <<= 1;
+  L.cap = fused ? kFilterCap / tp : 0;
   size_t o = 0;
-  L.ring = o;
-  o += (size_t)ns * stage_bytes;
-  L.score = o;
-  o += fused ? (size_t)kDecodeScoreCap * 4 : 0;
-  L.win = o;
-  o += fused ? 2048 * 4 : 0;
+  L.fbuf = o;  // per token: cap bits then cap indices; 2 * kFilterCap words in all
+  o += fused ? (size_t)kFilterCap * 8 : 0;
+  L.fstate = o;
+  o += fused ? align16(sizeof(FilterState) * kMaxFusedT) : 0;
   L.scratch = o;
-  o += fused ? ((sizeof(SelectScratch) + 15) & ~(size_t)15) : 0;
+  o += fused ? align16(sizeof(SelectScratch)) : 0;
+  L.sortv = o;
+  o += fused ? (size_t)(kMaxK + 2) * 8 : 0;
+  L.sortb = o;
+  o += fused ? (size_t)(kMaxK + 4) * 4 : 0;
   L.off = o;
-  o += ((size_t)(kDecodeMaxB + 1) * 4 + 15) & ~(size_t)15;
+  o += align16((size_t)(kDecodeMaxB + 1) * 4);
   L.bar = o;
   o += (size_t)2 * kMaxStages * 8;
   L.misc = o;
   o += 64;
+  o = (o + 127) & ~(size_t)127;
+  L.ring = o;  // the ring takes what is left
+  int ns = (int)(((size_t)kSmemMax - o) / stage_bytes);
+  if (ns > kMaxStages) ns = kMaxStages;
+  // About 128 KB in flight per SM streams at the HBM rate; deeper rings only
+  // add queueing.
+  const int ns_cap = (int)(kRingTargetBytes / stage_bytes);
+  if (ns > ns_cap && ns_cap >= kConsumerWarps) ns = ns_cap;
+  // A multiple of the consumer-warp count: slot s is then only ever consumed
+  // by warp s % 8, which waits on its full barrier's phases strictly in order
+  // (a waiter two phases ahead would see an old phase as complete).
+  ns -= ns % kConsumerWarps;
+  L.nstage = ns;
+  o += (size_t)ns * stage_bytes;
   L.total = o;
   return L;
 }
@@ -92,7 +109,19 @@ __device__ __forceinline__ int row_of(const int* s_off, int B, int gp) {
   return lo;
 }
 
-// Unpack 8 bf16 (one 16-byte chunk) to fp32.
+// Local page index in request b of the chunk boundary at global page x, snapped
+// down to a multiple of the stage size (or clamped to the row's ends).  Every
+// stage then starts at a request-local page index that is a multiple of 32, so
+// the arithmetic order of a page's score depends on the page alone, not on how
+// the batch was cut into chunks.
+__device__ __forceinline__ int snap_local(const int* s_off, int b, int x) {
+  const int len = s_off[b + 1] - s_off[b];
+  const int r = x - s_off[b];
+  if (r >= len) return len;
+  return r <= 0 ? 0 : (r & ~(kStagePages - 1));
+}
+
+// Unpack 8 bf16 (one 16-byte chunk) to fp32; element 2k is the low half of word k.
 __device__ __forceinline__ void unpack8(const uint4 v, float* f) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -102,15 +131,19 @@ __device__ __forceinline__ void unpack8(const uint4 v, float* f) {
   }
 }
 
-template <int LPP, int TT, bool FUSED>
+// D_T: head dim as a template constant (64, 128, 256), or 0 for any D % 8 == 0.
+template <int D_T, int TT, bool FUSED>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const DecodeLayout L = decode_layout(FUSED, a.D);
+  constexpr int CPL = D_T ? D_T / 32 : 8;  // 16-byte chunks per lane (max)
+  const int D = D_T ? D_T : a.D;
+  const DecodeLayout L = decode_layout(FUSED, D, a.T);
   unsigned char* ring = smem + L.ring;
-  uint32_t* s_score = reinterpret_cast<uint32_t*>(smem + L.score);
-  int* win_pos = reinterpret_cast<int*>(smem + L.win);
+  uint32_t* fbuf = reinterpret_cast<uint32_t*>(smem + L.fbuf);
+  FilterState* fst = reinterpret_cast<FilterState*>(smem + L.fstate);
   SelectScratch& sc = *reinterpret_cast<SelectScratch*>(smem + L.scratch);
-  uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem + L.scratch);
+  uint64_t* sortv = reinterpret_cast<uint64_t*>(smem + L.sortv);
+  uint32_t* sortb = reinterpret_cast<uint32_t*>(smem + L.sortb);
   int* s_off = reinterpret_cast<int*>(smem + L.off);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* empty = full + kMaxStages;
@@ -119,14 +152,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   int* s_flag = misc + 1;
   uint32_t* s_wsum = reinterpret_cast<uint32_t*>(misc + 4);  // 9 warp sums
 
-  constexpr int PPI = 32 / LPP;  // pages per warp instruction
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int G = gridDim.x;
   const int g = blockIdx.x;
-  const int B = a.B, T = a.T, N = a.N, D = a.D, Q = a.Q;
+  const int B = a.B, T = a.T, N = a.N, Q = a.Q;
   const int nst = L.nstage;
+  const int cap = L.cap;
   const uint32_t page_bytes = (uint32_t)D * 2;
   const uint32_t stage_bytes = page_bytes * kStagePages;
 
@@ -167,43 +200,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   }
   __syncthreads();
   const int P = s_off[B];
-  int Lc;
-  if (FUSED) {
-    Lc = (P + G - 1) / G;
-    Lc = Lc < kLMin ? kLMin : Lc;
-    const int lmax = kDecodeScoreCap / T;
-    Lc = Lc > lmax ? lmax : Lc;
-  } else {
-    Lc = (P + G - 1) / G;
-    Lc = Lc < 1 ? 1 : Lc;
-  }
+  int Lc = (P + G - 1) / G;
+  if (FUSED) Lc = Lc < kLMin ? kLMin : Lc;
+  Lc = Lc < 1 ? 1 : Lc;
   const int nchunks = (P + Lc - 1) / Lc;
 
   // ------------------------------------------------------------------ producer
+  // Lanes 0..kProducerLanes-1 issue the stages round-robin (stage k by lane
+  // k % kProducerLanes): one issuing thread alone caps the copy rate well
+  // below HBM bandwidth.  The ring depth is a multiple of kProducerLanes, so a
+  // slot is always refilled by the same lane, in order.
   if (warp == kConsumerWarps) {
-    if (lane == 0) {
+    if (lane < kProducerLanes) {
       const uint64_t pol = policy_evict_first();
       uint32_t stage = 0;
       for (int j = g; j < nchunks; j += G) {
         const int cb = j * Lc, ce = min(cb + Lc, P);
-        int b = row_of(s_off, B, cb);
-        for (int gp = cb; gp < ce;) {
-          while (s_off[b + 1] <= gp) ++b;
-          const int se = min(ce, s_off[b + 1]);
-          const int p0 = gp - s_off[b];
-          const int np = se - gp;
+        const int b_last = row_of(s_off, B, ce - 1);
+        for (int b = row_of(s_off, B, cb); b <= b_last; ++b) {
+          if (s_off[b + 1] == s_off[b]) continue;
+          const int p0 = snap_local(s_off, b, cb);
+          const int np = snap_local(s_off, b, ce) - p0;
           const uint16_t* src = a.c + (int64_t)b * a.ldc_b + (int64_t)p0 * D;
           for (int sp = 0; sp < np; sp += kStagePages, ++stage) {
+            if ((int)(stage % kProducerLanes) != lane) continue;
             const int slot = (int)(stage % (uint32_t)nst);
             const uint32_t round = stage / (uint32_t)nst;
             if (round > 0) mbar_wait_bounded(&empty[slot], (round - 1) & 1, s_abort, a.status);
             if (*s_abort) continue;
             const uint32_t bytes = (uint32_t)min(kStagePages, np - sp) * page_bytes;
             mbar_arrive_expect_tx(&full[slot], bytes);
+#ifdef IDX_NO_L2_HINT
+            bulk_g2s_nohint(ring + (size_t)slot * stage_bytes, src + (int64_t)sp * D, bytes,
+                            &full[slot]);
+            (void)pol;
+#else
             bulk_g2s(ring + (size_t)slot * stage_bytes, src + (int64_t)sp * D, bytes, &full[slot],
                      pol);
+#endif
           }
-          gp = se;
         }
       }
     }
@@ -212,34 +247,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
 
   // ------------------------------------------------------------------ consumers
   if (!FUSED) {
-    // -inf for the padded pages p >= len[b] of every token row, balanced over CTAs.
-    const int64_t per_tok_total = (int64_t)B * N - P;
-    const int64_t tot = per_tok_total * T;
-    const int64_t beg = tot * g / G, end = tot * (g + 1) / G;
-    if (beg < end) {
-      // first request whose padding extends past beg
-      int lo = 0, hi = B - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        const int64_t pad_next = (int64_t)T * ((int64_t)(mid + 1) * N - s_off[mid + 1]);
-        if (pad_next > beg) hi = mid;
-        else lo = mid + 1;
-      }
-      int64_t x = beg;
-      for (int b = lo; x < end && b < B; ++b) {
-        const int lb = s_off[b + 1] - s_off[b];
-        const int64_t per = N - lb;
-        const int64_t rb = (int64_t)T * ((int64_t)b * N - s_off[b]);
-        const int64_t re = rb + per * T;
-        const int64_t e = end < re ? end : re;
-        for (int64_t y = x + tid; y < e; y += kConsumers) {
-          const int64_t r = y - rb;
-          const int t = (int)(r / per);
-          const int p = lb + (int)(r % per);
-          a.scores[((int64_t)b * T + t) * N + p] = __uint_as_float(kNegInfBits);
-        }
-        if (e > x) x = e;
-      }
+    // -inf for the padded pages p >= len[b] of every token row: rows are cut
+    // into 4096-entry pieces dealt round-robin to the CTAs.
+    constexpr int kPiece = 4096;
+    const int ppr = (N + kPiece - 1) / kPiece;  // pieces per row
+    const int64_t npieces = (int64_t)B * T * ppr;
+    for (int64_t pc = g; pc < npieces; pc += G) {
+      const int rowi = (int)(pc / ppr);
+      const int b = rowi / T;
+      const int lb = s_off[b + 1] - s_off[b];
+      const int p_lo = max(lb, (int)(pc - (int64_t)rowi * ppr) * kPiece);
+      const int p_hi = min(N, (int)(pc - (int64_t)rowi * ppr) * kPiece + kPiece);
+      float* dst = a.scores + (int64_t)rowi * N;
+      for (int p = p_lo + tid; p < p_hi; p += kConsumers) dst[p] = __uint_as_float(kNegInfBits);
     }
   } else {
     // Rows with no valid page: their output is all padding.
@@ -253,181 +273,217 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
     }
   }
 
-  const int nchunks_d = D >> 3;  // 16-byte chunks per page
-  const int chunk_id = lane & (LPP - 1);
-  const int sub = lane / LPP;
-  const int my_page = chunk_id * PPI + sub;  // page this lane holds after the butterfly
+  // Lane geometry: lane = 4 * pg + c4; page-group pg (0..7) of each 8-page
+  // instruction, lane c4 (0..3) within the page.
+  const int pg = lane >> 2;
+  const int c4 = lane & 3;
+  const int nchunk = D >> 3;  // 16-byte chunks per page
+  const int cpl = D_T ? CPL : (nchunk + 3) / 4;
+  uint32_t lane_off[CPL];
+  bool chunk_ok[CPL];
+  int chunk_of[CPL];
+#pragma unroll
+  for (int jj = 0; jj < CPL; ++jj) {
+    const int ch = c4 + 4 * ((jj + pg) % cpl);
+    chunk_of[jj] = ch;
+    chunk_ok[jj] = (jj < cpl) && (ch < nchunk);
+    lane_off[jj] = (uint32_t)pg * page_bytes + (uint32_t)ch * 16u;
+  }
+  const int my_page = c4 * 8 + pg;  // page this lane holds after the butterfly
+  // Check the filters every `rounds` rounds of 8 stages (a round appends at
+  // most 256 entries per token), and compact a token's filter once it holds a
+  // few K entries (early, so the threshold rises fast) and always before the
+  // next check could overflow it.
+  const int rounds = FUSED ? max(1, min(4, (cap - a.K) / kConsumers)) : 1;
+  const int compact_at = min(cap - rounds * kConsumers, max(4 * a.K, 1024));
+  const int check_period = rounds * kConsumerWarps;
+  const bool q_resident = (T <= TT);
+
+  float qr[TT][CPL][8];
   uint32_t stage = 0;
-  int cur_b = -1;
-  float qs[TT][8];
 
   for (int j = g; j < nchunks; j += G) {
     const int cb = j * Lc, ce = min(cb + Lc, P);
-    int b = row_of(s_off, B, cb);
-    for (int gp = cb; gp < ce;) {
-      while (s_off[b + 1] <= gp) ++b;
-      const int se = min(ce, s_off[b + 1]);
-      const int p0 = gp - s_off[b];
-      const int np = se - gp;
-      const int local = gp - cb;
+    const int b_last = row_of(s_off, B, ce - 1);
+    for (int b = row_of(s_off, B, cb); b <= b_last; ++b) {
+      if (s_off[b + 1] == s_off[b]) continue;
+      const int p0 = snap_local(s_off, b, cb);
+      const int np = snap_local(s_off, b, ce) - p0;  // may be 0
+      if (FUSED) {
+        if (tid < T) filter_reset(fst[tid]);
+        group_sync(kConsumers);
+      }
       for (int sp = 0; sp < np; sp += kStagePages, ++stage) {
-        if ((int)(stage % kConsumerWarps) != warp) continue;
-        const int slot = (int)(stage % (uint32_t)nst);
-        mbar_wait_bounded(&full[slot], (stage / (uint32_t)nst) & 1, s_abort, a.status);
-        const unsigned char* sb = ring + (size_t)slot * stage_bytes;
-        const int n_here = min(kStagePages, np - sp);
-        for (int t0 = 0; t0 < T; t0 += TT) {
-          // pre-summed query of tokens t0..t0+TT-1 for this lane's 8 dims
-          if (b != cur_b || T > TT) {
-#pragma unroll
-            for (int t = 0; t < TT; ++t) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) qs[t][e] = 0.f;
-              if (t0 + t < T && chunk_id < nchunks_d) {
-                const uint16_t* qp = a.q + (((int64_t)b * T + t0 + t) * Q) * D + chunk_id * 8;
-                for (int h = 0; h < Q; ++h) {
-                  float f[8];
-                  unpack8(*reinterpret_cast<const uint4*>(qp + (int64_t)h * D), f);
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) qs[t][e] += f[e];
-                }
-              }
-            }
-            cur_b = b;
-          }
-          float acc[TT][LPP];
-#pragma unroll
-          for (int t = 0; t < TT; ++t)
-#pragma unroll
-            for (int i = 0; i < LPP; ++i) acc[t][i] = 0.f;
-#pragma unroll
-          for (int i = 0; i < LPP; ++i) {
-            const int page = i * PPI + sub;
-            if (page < n_here && chunk_id < nchunks_d) {
-              const uint4 v = *reinterpret_cast<const uint4*>(sb + (size_t)page * page_bytes +
-                                                              chunk_id * 16);
-              float f[8];
-              unpack8(v, f);
+        if ((int)(stage % kConsumerWarps) == warp) {
+          const int slot = (int)(stage % (uint32_t)nst);
+          mbar_wait_bounded(&full[slot], (stage / (uint32_t)nst) & 1, s_abort, a.status);
+          const unsigned char* sb = ring + (size_t)slot * stage_bytes;
+          const int n_here = min(kStagePages, np - sp);
+          for (int t0 = 0; t0 < T; t0 += TT) {
+            if (!q_resident || sp < kConsumerWarps * kStagePages) {
+              // pre-summed query chunks (first stage of this warp in the
+              // segment, or every stage when the tokens do not fit registers)
 #pragma unroll
               for (int t = 0; t < TT; ++t)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[t][i] = fmaf(qs[t][e], f[e], acc[t][i]);
-            }
-          }
-          // transposed butterfly over the LPP lanes of a page
+                for (int jj = 0; jj < CPL; ++jj) {
 #pragma unroll
-          for (int m = LPP / 2; m >= 1; m >>= 1) {
-            const bool upper = (lane & m) != 0;
+                  for (int e = 0; e < 8; ++e) qr[t][jj][e] = 0.f;
+                  if (t0 + t < T && chunk_ok[jj]) {
+                    const uint16_t* qp =
+                        a.q + ((int64_t)b * T + t0 + t) * Q * D + chunk_of[jj] * 8;
+                    for (int h = 0; h < Q; ++h) {
+                      float f[8];
+                      unpack8(*reinterpret_cast<const uint4*>(qp + (int64_t)h * D), f);
+#pragma unroll
+                      for (int e = 0; e < 8; ++e) qr[t][jj][e] += f[e];
+                    }
+                  }
+                }
+            }
+            float acc[TT][4];
+#pragma unroll
+            for (int t = 0; t < TT; ++t)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) acc[t][i] = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < CPL; ++jj) {
+              if (D_T || chunk_ok[jj]) {
+                uint4 v[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                  v[i] = *reinterpret_cast<const uint4*>(sb + lane_off[jj] + i * 8 * page_bytes);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float f[8];
+                  unpack8(v[i], f);
+#pragma unroll
+                  for (int t = 0; t < TT; ++t)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[t][i] = fmaf(qr[t][jj][e], f[e], acc[t][i]);
+                }
+              }
+            }
+            // butterfly over the 4 lanes of a page: lane c4 ends with group c4's sum
+            const bool u2 = (lane & 2) != 0, u1 = (lane & 1) != 0;
 #pragma unroll
             for (int t = 0; t < TT; ++t) {
 #pragma unroll
-              for (int jj = 0; jj < m; ++jj) {
-                const float send = upper ? acc[t][jj] : acc[t][jj + m];
-                const float keep = upper ? acc[t][jj + m] : acc[t][jj];
-                acc[t][jj] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, m);
+              for (int jj = 0; jj < 2; ++jj) {
+                const float send = u2 ? acc[t][jj] : acc[t][jj + 2];
+                const float keep = u2 ? acc[t][jj + 2] : acc[t][jj];
+                acc[t][jj] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 2);
               }
+              const float send = u1 ? acc[t][0] : acc[t][1];
+              const float keep = u1 ? acc[t][1] : acc[t][0];
+              acc[t][0] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 1);
             }
-          }
-          if (my_page < n_here) {
+            const bool mine = my_page < n_here;
 #pragma unroll
             for (int t = 0; t < TT; ++t) {
               if (t0 + t < T) {
                 if (FUSED) {
-                  s_score[(t0 + t) * Lc + local + sp + my_page] = __float_as_uint(acc[t][0]);
-                } else {
+                  uint32_t* fb = fbuf + (t0 + t) * 2 * cap;
+                  filter_offer(fst[t0 + t], fb, fb + cap, __float_as_uint(acc[t][0]),
+                               (uint32_t)(p0 + sp + my_page), mine);
+                } else if (mine) {
                   a.scores[((int64_t)b * T + t0 + t) * N + p0 + sp + my_page] = acc[t][0];
                 }
               }
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[slot]);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (FUSED && ((stage % check_period) == check_period - 1 || sp + kStagePages >= np)) {
+          group_sync(kConsumers);  // this round's offers are complete
+          for (int t = 0; t < T; ++t)
+            if (fst[t].count > compact_at)
+              filter_compact<kConsumers>(fst[t], fbuf + t * 2 * cap, fbuf + t * 2 * cap + cap,
+                                         a.K, sc);
+        }
       }
       if (FUSED) {
-        group_sync(kConsumers);  // every stage of this row segment is scored
         const int j0 = s_off[b] / Lc;
         const int j1 = (s_off[b + 1] - 1) / Lc;
-        const bool single = (j0 == j1);
         for (int t = 0; t < T; ++t) {
-          const uint32_t* row = s_score + t * Lc + local;
-          const int kk = block_select<kConsumers>(row, np, a.K, win_pos, sc);
+          uint32_t* fb = fbuf + t * 2 * cap;
+          uint32_t* fi = fb + cap;
+          filter_compact<kConsumers>(fst[t], fb, fi, a.K, sc);
+          const int kk = fst[t].count;
           const int64_t orow = (int64_t)b * T + t;
-          if (single) {
-            sort_and_write<kConsumers>(row, nullptr, p0, win_pos, kk, a.K, sortbuf,
-                                       a.idx_out + orow * a.K,
+          if (j0 == j1) {
+            sort_and_write<kConsumers>(fb, fi, kk, a.K, sortv, sortb, a.idx_out + orow * a.K,
                                        a.val_out ? a.val_out + orow * a.K : nullptr);
           } else {
             const int64_t slot = (int64_t)(j + b) * T + t;
-            uint32_t* cbits = a.cand_bits + slot * a.slot_stride;
-            int32_t* cidx = a.cand_idx + slot * a.slot_stride;
-            for (int k = tid; k < kk; k += kConsumers) {
-              const int p = win_pos[k];
-              cbits[k] = row[p];
-              cidx[k] = p0 + p;
-            }
-            if (tid == 0) a.cand_cnt[slot] = kk;
+            publish_candidates<kConsumers>(fb, fi, kk, a.K, fst[t].thr,
+                                           a.cand_bits + slot * a.slot_stride,
+                                           a.cand_idx + slot * a.slot_stride, a.row_thr + orow);
           }
         }
-        if (!single && arrive_last<kConsumers>(a.arrive + b, j1 - j0 + 1, s_flag)) {
-          const int cap = kDecodeScoreCap / 2;
-          uint32_t* m_bits = s_score;
-          int32_t* m_idx = reinterpret_cast<int32_t*>(s_score + cap);
+        if (j0 != j1 && arrive_last<kConsumers>(a.arrive + b, j1 - j0 + 1, s_flag)) {
           for (int t = 0; t < T; ++t) {
             const int64_t orow = (int64_t)b * T + t;
             merge_candidates<kConsumers>(
                 j1 - j0 + 1, [=](int i) { return (int64_t)(j0 + i + b) * T + t; }, a.cand_bits,
-                a.cand_idx, a.cand_cnt, a.slot_stride, a.K, cap, m_bits, m_idx, win_pos, sc,
-                sortbuf, a.idx_out + orow * a.K, a.val_out ? a.val_out + orow * a.K : nullptr);
+                a.cand_idx, a.slot_stride, a.K, a.row_thr + orow, fst[0], fbuf,
+                fbuf + kFilterCap, kFilterCap, sc, sortv, sortb, a.idx_out + orow * a.K,
+                a.val_out ? a.val_out + orow * a.K : nullptr);
           }
         }
+        group_sync(kConsumers);
       }
-      gp = se;
     }
   }
 }
 
 int decode_grid(int num_sms) { return num_sms; }
 
-int64_t decode_fused_slots(int64_t B, int64_t T, int64_t N, int grid) {
-  // The kernel's chunk length is clamp(ceil(P/grid), kLMin, floor(cap/T)), so
-  // chunks <= max(grid, ceil(B*N / floor(cap/T))); the pair (chunk j,
-  // request b) owns slot (j + b) for each of its T tokens.
-  const int64_t lmax = kDecodeScoreCap / T;
-  int64_t chunks = (B * N + lmax - 1) / lmax;
-  if (chunks < grid) chunks = grid;
-  return (chunks + 1 + B) * T;
+int decode_fused_max_k(int T) {
+  if (T > kMaxFusedT) return 0;
+  int tp = 1;
+  while (tp < T) tp <<= 1;
+  const int k = kFilterCap / tp - kConsumers;
+  return k < kMaxK ? k : kMaxK;
 }
 
-template <int LPP, int TT, bool FUSED>
+int64_t decode_fused_slots(int64_t B, int64_t T, int64_t N, int grid) {
+  // The fused chunk length is max(ceil(P/grid), kLMin), so there are at most
+  // `grid` chunks; the pair (chunk j, request b) owns slot (j + b) per token.
+  (void)N;
+  return ((int64_t)grid + 1 + B) * T;
+}
+
+template <int D_T, int TT, bool FUSED>
 static cudaError_t launch_one(const DecodeArgs& a, int grid, cudaStream_t stream) {
-  const DecodeLayout L = decode_layout(FUSED, a.D);
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<LPP, TT, FUSED>,
+  const DecodeLayout L = decode_layout(FUSED, a.D, a.T);
+  if (L.nstage < kConsumerWarps || L.total > (size_t)kSmemMax) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<D_T, TT, FUSED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
-  decode_kernel<LPP, TT, FUSED><<<grid, kDecodeThreads, L.total, stream>>>(a);
+  decode_kernel<D_T, TT, FUSED><<<grid, kDecodeThreads, L.total, stream>>>(a);
   return cudaGetLastError();
 }
 
-template <int LPP, bool FUSED>
+template <int D_T, bool FUSED>
 static cudaError_t launch_tt(const DecodeArgs& a, int grid, cudaStream_t stream) {
-  // register budget: TT * LPP accumulators
-  if (a.T == 1) return launch_one<LPP, 1, FUSED>(a, grid, stream);
-  if (a.T == 2 || LPP == 32) return launch_one<LPP, 2, FUSED>(a, grid, stream);
-  return launch_one<LPP, 4, FUSED>(a, grid, stream);
+  if (a.T == 1) return launch_one<D_T, 1, FUSED>(a, grid, stream);
+  return launch_one<D_T, 2, FUSED>(a, grid, stream);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream) {
   const int grid = decode_grid(num_sms);
-  const int chunks = a.D / 8;
   if (fused) {
-    if (chunks <= 8) return launch_tt<8, true>(a, grid, stream);
-    if (chunks <= 16) return launch_tt<16, true>(a, grid, stream);
-    return launch_tt<32, true>(a, grid, stream);
+    if (a.D == 128) return launch_tt<128, true>(a, grid, stream);
+    if (a.D == 64) return launch_tt<64, true>(a, grid, stream);
+    if (a.D == 256) return launch_tt<256, true>(a, grid, stream);
+    return launch_tt<0, true>(a, grid, stream);
   }
-  if (chunks <= 8) return launch_tt<8, false>(a, grid, stream);
-  if (chunks <= 16) return launch_tt<16, false>(a, grid, stream);
-  return launch_tt<32, false>(a, grid, stream);
+  if (a.D == 128) return launch_tt<128, false>(a, grid, stream);
+  if (a.D == 64) return launch_tt<64, false>(a, grid, stream);
+  if (a.D == 256) return launch_tt<256, false>(a, grid, stream);
+  return launch_tt<0, false>(a, grid, stream);
 }
 
 }  // namespace idx

@@ -6,6 +6,8 @@
 
 namespace idx {
 
+constexpr int kMaxK = 2048;  // the ABI's IDX_MAX_K
+
 // ---------------------------------------------------------------- top-K select
 struct TopkArgs {
   const float* scores;
@@ -21,7 +23,7 @@ struct TopkArgs {
   float* val_out;  // may be null
   uint32_t* cand_bits;
   int32_t* cand_idx;
-  int32_t* cand_cnt;
+  unsigned long long* row_thr;  // per-row shared thresholds, zero between calls
   int32_t* arrive;  // per-row arrival counters, zero between calls
   int* status;
 };
@@ -42,16 +44,17 @@ struct DecodeArgs {
   float* val_out;   // fused mode, may be null
   uint32_t* cand_bits;
   int32_t* cand_idx;
-  int32_t* cand_cnt;
-  int64_t slot_stride;  // entries per candidate slot (>= K)
-  int32_t* arrive;      // per-request arrival counters, zero between calls
+  int64_t slot_stride;          // entries per candidate slot (>= K)
+  unsigned long long* row_thr;  // per-row shared thresholds, zero between calls
+  int32_t* arrive;              // per-request arrival counters, zero between calls
   int* status;
 };
 constexpr int kDecodeMaxB = 1024;       // requests per launch (host splits larger batches)
 constexpr int kDecodeMaxTFused = 4;     // tokens per request on the fused CUDA-core path
-constexpr int kDecodeScoreCap = 16384;  // fused: fp32 scores a CTA keeps on chip
 // Candidate slots a fused launch of B requests x T tokens can use.
 int64_t decode_fused_slots(int64_t B, int64_t T, int64_t N, int grid);
+// Largest K the fused CUDA-core path takes for T tokens (its on-chip filter).
+int decode_fused_max_k(int T);
 int decode_grid(int num_sms);
 cudaError_t launch_decode(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream);
 

@@ -1,39 +1,42 @@
 // topk.cu -- standalone exact top-K over fp32 score rows ("Iterate Topk",
 // opening description: given per-segment scores, return the top-K indices).
 //
-// Grid (chunks, rows).  Each CTA loads one chunk of a row into shared memory
-// with coalesced 16-byte loads, selects the chunk's exact top-K' with the
-// block radix select, and either writes the final row directly (a row that
-// fits one chunk) or publishes its candidates; the last CTA of the row to
-// arrive merges them.  Short rows therefore take one CTA and one HBM read;
-// long rows spread over many SMs and still read every score exactly once.
+// Grid (chunks, rows).  Each CTA streams one chunk of a row from HBM with
+// coalesced 16-byte loads (one round prefetched ahead) and offers every
+// element to the exact online top-K filter of select.cuh; rounds are visited
+// in bit-reversed order, so a row sorted ascending or descending still raises
+// the threshold early.  A row that fits one chunk is sorted and written by
+// its CTA; otherwise each chunk publishes its K' candidates and the last CTA
+// of the row to arrive merges them.  Every score is read from HBM once.
 #include "common.cuh"
 #include "kernels.h"
-#include "merge.cuh"
+#include "select.cuh"
 
 namespace idx {
 
-constexpr int kTopkThreads = 512;
-constexpr int kTopkMaxChunk = 8192;
+constexpr int kTopkThreads = 256;
+constexpr int kTopkMaxChunk = 16384;
 constexpr int kTopkMinChunk = 2048;
+constexpr int kTopkVec = 4;                               // float4 loads per thread per round
+constexpr int kTopkRound = kTopkThreads * 4 * kTopkVec;  // elements per round
 
 struct TopkLayout {
-  size_t bits, gidx, win, scratch, flag, total;
+  size_t fbuf, fstate, scratch, sortv, sortb, flag, total;
 };
 
-__host__ __device__ inline TopkLayout topk_layout(int cap, int K) {
+__host__ __device__ inline TopkLayout topk_layout() {
   TopkLayout L;
   size_t o = 0;
-  L.bits = o;
-  o += (size_t)cap * 4;
-  L.gidx = o;
-  o += (size_t)cap * 4;
-  L.win = o;
-  o += ((size_t)K * 4 + 15) & ~(size_t)15;
+  L.fbuf = o;
+  o += (size_t)kFilterCap * 8;
+  L.fstate = o;
+  o += 16;
   L.scratch = o;
-  size_t sortb = (size_t)next_pow2(K) * 8;
-  o += (sizeof(SelectScratch) > sortb ? sizeof(SelectScratch) : sortb);
-  o = (o + 15) & ~(size_t)15;
+  o += (sizeof(SelectScratch) + 15) & ~(size_t)15;
+  L.sortv = o;
+  o += (size_t)(kMaxK + 2) * 8;
+  L.sortb = o;
+  o += (size_t)(kMaxK + 4) * 4;
   L.flag = o;
   o += 16;
   L.total = o;
@@ -51,90 +54,119 @@ __device__ __forceinline__ int clamp_len(const int32_t* lengths, int r, int N, i
   return l;
 }
 
-// Copy n fp32 bit patterns from global memory into shared memory.
-template <int NT>
-__device__ __forceinline__ void load_bits(uint32_t* dst, const float* src, int n) {
-  const uint32_t* s = reinterpret_cast<const uint32_t*>(src);
-  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
-    const int n4 = n >> 2;
-    const uint4* s4 = reinterpret_cast<const uint4*>(s);
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
-    constexpr int U = 4;
-    for (int base = threadIdx.x; base < n4; base += NT * U) {
-      uint4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (base + u * NT < n4) v[u] = __ldcs(s4 + base + u * NT);
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        if (base + u * NT < n4) d4[base + u * NT] = v[u];
-    }
-    for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) dst[i] = __ldcs(s + i);
-  } else {
-    for (int i = threadIdx.x; i < n; i += NT) dst[i] = __ldcs(s + i);
-  }
+__device__ __forceinline__ uint32_t bit_reverse(uint32_t x, int bits) {
+  return bits ? (__brev(x) >> (32 - bits)) : 0u;
 }
 
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_chunk_kernel(const TopkArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  const int cap = a.chunk > 2 * a.K ? a.chunk : 2 * a.K;
-  const TopkLayout L = topk_layout(cap, a.K);
-  uint32_t* s_bits = reinterpret_cast<uint32_t*>(smem + L.bits);
-  int32_t* s_idx = reinterpret_cast<int32_t*>(smem + L.gidx);
-  int* win_pos = reinterpret_cast<int*>(smem + L.win);
+  const TopkLayout L = topk_layout();
+  uint32_t* fb = reinterpret_cast<uint32_t*>(smem + L.fbuf);
+  uint32_t* fi = fb + kFilterCap;
+  FilterState& fs = *reinterpret_cast<FilterState*>(smem + L.fstate);
   SelectScratch& sc = *reinterpret_cast<SelectScratch*>(smem + L.scratch);
-  uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem + L.scratch);
+  uint64_t* sortv = reinterpret_cast<uint64_t*>(smem + L.sortv);
+  uint32_t* sortb = reinterpret_cast<uint32_t*>(smem + L.sortb);
   int* s_flag = reinterpret_cast<int*>(smem + L.flag);
 
+  const int tid = threadIdx.x;
   const int row = blockIdx.y;
   const int ch = blockIdx.x;
-  const int len =
-      clamp_len(a.lengths, row / a.len_div, a.N, a.status, ch == 0 && threadIdx.x == 0);
+  const int len = clamp_len(a.lengths, row / a.len_div, a.N, a.status, ch == 0 && tid == 0);
   const int nch = len > 0 ? (len + a.chunk - 1) / a.chunk : 1;
   if (ch >= nch) return;
   const int c0 = ch * a.chunk;
   const int n = max(0, min(a.chunk, len - c0));
+  const float* src = a.scores + (int64_t)row * a.lds + c0;
+  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
 
   int32_t* io = a.idx_out + (int64_t)row * a.K;
   float* vo = a.val_out ? a.val_out + (int64_t)row * a.K : nullptr;
 
-  load_bits<NT>(s_bits, a.scores + (int64_t)row * a.lds + c0, n);
+  if (tid == 0) filter_reset(fs);
   group_sync(NT);
-  const int kk = block_select<NT>(s_bits, n, a.K, win_pos, sc);
+  // compact once the filter holds a few K entries (the threshold then rises
+  // early), and always before the next 4*NT offers could overflow it
+  const int compact_at = min(kFilterCap - 4 * NT, max(4 * a.K, 1024));
+
+  // Round r covers elements [r * kTopkRound, (r+1) * kTopkRound) of the chunk;
+  // thread tid loads float4 number tid + u * NT (u < kTopkVec) of the round.
+  const int rounds = (n + kTopkRound - 1) / kTopkRound;
+  int rbits = 0;
+  while ((1 << rbits) < rounds) ++rbits;
+  uint4 cur[kTopkVec], nxt[kTopkVec];
+  int seq = 0;
+  // next round index in bit-reversed order, skipping indices past `rounds`
+  auto next_round = [&]() {
+    while (seq < (1 << rbits)) {
+      const int cand = (int)bit_reverse((uint32_t)seq++, rbits);
+      if (cand < rounds) return cand;
+    }
+    return -1;
+  };
+  auto load_round = [&](int r, uint4 (&buf)[kTopkVec]) {
+#pragma unroll
+    for (int u = 0; u < kTopkVec; ++u) {
+      const int e0 = r * kTopkRound + 4 * (tid + u * NT);
+      if (vec && e0 + 3 < n) {
+        buf[u] = __ldcs(reinterpret_cast<const uint4*>(src + e0));
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          w[k] = (e0 + k < n) ? __float_as_uint(__ldcs(src + e0 + k)) : kNegInfBits;
+        buf[u] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  };
+  int r = rounds > 0 ? next_round() : -1;
+  if (r >= 0) load_round(r, cur);
+  while (r >= 0) {
+    const int rn = next_round();
+    if (rn >= 0) load_round(rn, nxt);
+#pragma unroll
+    for (int u = 0; u < kTopkVec; ++u) {
+      const int e0 = r * kTopkRound + 4 * (tid + u * NT);
+      const uint32_t w[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        filter_offer(fs, fb, fi, w[k], (uint32_t)(c0 + e0 + k), e0 + k < n);
+      group_sync(NT);
+      if (fs.count > compact_at) filter_compact<NT>(fs, fb, fi, a.K, sc);
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkVec; ++u) cur[u] = nxt[u];
+    r = rn;
+  }
+  group_sync(NT);
+  filter_compact<NT>(fs, fb, fi, a.K, sc);
+  const int kk = fs.count;
   if (nch == 1) {
-    sort_and_write<NT>(s_bits, nullptr, 0, win_pos, kk, a.K, sortbuf, io, vo);
+    sort_and_write<NT>(fb, fi, kk, a.K, sortv, sortb, io, vo);
     return;
   }
   const int64_t slot = (int64_t)row * a.max_chunks + ch;
-  uint32_t* cb = a.cand_bits + slot * a.slot_stride;
-  int32_t* ci = a.cand_idx + slot * a.slot_stride;
-  for (int k = threadIdx.x; k < kk; k += NT) {
-    const int p = win_pos[k];
-    cb[k] = s_bits[p];
-    ci[k] = c0 + p;
-  }
-  if (threadIdx.x == 0) a.cand_cnt[slot] = kk;
+  publish_candidates<NT>(fb, fi, kk, a.K, fs.thr, a.cand_bits + slot * a.slot_stride,
+                         a.cand_idx + slot * a.slot_stride, a.row_thr + row);
   if (!arrive_last<NT>(a.arrive + row, nch, s_flag)) return;
   const int64_t base = (int64_t)row * a.max_chunks;
   merge_candidates<NT>(
-      nch, [base](int i) { return base + i; }, a.cand_bits, a.cand_idx, a.cand_cnt,
-      a.slot_stride, a.K, cap, s_bits, s_idx, win_pos, sc, sortbuf, io, vo);
+      nch, [base](int i) { return base + i; }, a.cand_bits, a.cand_idx, a.slot_stride, a.K,
+      a.row_thr + row, fs, fb, fi, kFilterCap, sc, sortv, sortb, io, vo);
 }
 
 int topk_plan_chunk(int rows, int N, int K, int num_sms) {
+  (void)K;
   int chunk = kTopkMaxChunk;
-  const int floor_chunk = kTopkMinChunk > 2 * K ? kTopkMinChunk : next_pow2(2 * K);
-  while (chunk > floor_chunk &&
-         (int64_t)rows * ((N + chunk - 1) / chunk) < 2 * (int64_t)num_sms)
+  while (chunk > kTopkMinChunk &&
+         (int64_t)rows * ((N + chunk - 1) / chunk) < 3 * (int64_t)num_sms)
     chunk >>= 1;
-  if (chunk < floor_chunk) chunk = floor_chunk;
   return chunk;
 }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream) {
-  const int cap = a.chunk > 2 * a.K ? a.chunk : 2 * a.K;
-  const TopkLayout L = topk_layout(cap, a.K);
+  const TopkLayout L = topk_layout();
   cudaError_t e = cudaFuncSetAttribute(topk_chunk_kernel<kTopkThreads>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;

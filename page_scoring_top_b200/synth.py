@@ -73,9 +73,10 @@ def uniform24(x: np.ndarray) -> np.ndarray:
 
 
 def normal(seed: int, stream: int, start: int, count: int) -> np.ndarray:
-    """``count`` standard normals (double) starting at normal number ``start``
-    (``start`` even: normals come in Box-Muller pairs)."""
-    assert start % 2 == 0
+    """``count`` standard normals (double): numbers start .. start+count-1 of
+    the stream's normal sequence (pair k = draws 2k, 2k+1)."""
+    if start % 2:
+        return normal(seed, stream, start - 1, count + 1)[1:]
     npairs = (count + 1) // 2
     out = np.empty(2 * npairs, np.float64)
     for off in range(0, npairs, _CHUNK // 2):

@@ -26,6 +26,7 @@ def test_counter_based_slices():
     assert np.array_equal(synth.u64(3, 5, 400, 100), full[400:500])
     nfull = synth.normal(3, 5, 0, 1000)
     assert np.array_equal(synth.normal(3, 5, 200, 300), nfull[200:500])
+    assert np.array_equal(synth.normal(3, 5, 201, 299), nfull[201:500])   # odd start
     assert not np.array_equal(synth.u64(3, 6, 0, 10), full[:10])   # streams differ
 
 
