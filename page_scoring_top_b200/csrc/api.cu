@@ -101,19 +101,23 @@ int run_topk(idx_ctx* ctx, const float* scores, const int32_t* lengths, int len_
 int run_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths, int B,
               int T, int Q, int D, int N, int64_t ldc_b, float* scores, cudaStream_t stream) {
   if (idx::prefill_supported(T, Q, D, ldc_b)) {
-    idx::PrefillArgs p{};
-    p.q = q;
-    p.c = c;
-    p.lengths = lengths;
-    p.B = B;
-    p.T = T;
-    p.Q = Q;
-    p.D = D;
-    p.N = N;
-    p.ldc_b = ldc_b;
-    p.scores = scores;
-    p.status = ctx->status;
-    return status_of(idx::launch_prefill(p, ctx->num_sms, stream));
+    for (int b0 = 0; b0 < B; b0 += idx::kPrefillMaxB) {
+      idx::PrefillArgs p{};
+      p.q = q + (int64_t)b0 * T * Q * D;
+      p.c = c + (int64_t)b0 * ldc_b;
+      p.lengths = lengths ? lengths + b0 : nullptr;
+      p.B = std::min(idx::kPrefillMaxB, B - b0);
+      p.T = T;
+      p.Q = Q;
+      p.D = D;
+      p.N = N;
+      p.ldc_b = ldc_b;
+      p.scores = scores + (int64_t)b0 * T * N;
+      p.status = ctx->status;
+      const int rc = status_of(idx::launch_prefill(p, ctx->num_sms, stream));
+      if (rc != IDX_OK) return rc;
+    }
+    return IDX_OK;
   }
   for (int b0 = 0; b0 < B; b0 += idx::kDecodeMaxB) {
     const int nb = std::min(idx::kDecodeMaxB, B - b0);

@@ -68,6 +68,7 @@ struct PrefillArgs {
   float* scores;  // [B][T][N]
   int* status;
 };
+constexpr int kPrefillMaxB = 256;  // requests per launch (host splits larger batches)
 bool prefill_supported(int T, int Q, int D, int64_t ldc_b);
 cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t stream);
 
