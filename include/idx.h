@@ -132,6 +132,27 @@ IDX_API const char* idx_strerror(int code);
 /* Number of SMs the context sizes its persistent grids for (0 if ctx is NULL). */
 IDX_API int idx_num_sms(const idx_ctx* ctx);
 
+/*
+ * topk_select without a context, for callers that cannot allocate device
+ * memory: code running while a CUDA graph is captured, serving engines that
+ * plan all device memory up front, plugin hosts that provide no allocator.
+ * The pages have no counterpart of this call; it exists for those callers.
+ *
+ * Same arguments, result and error codes as topk_select, on the calling
+ * thread's current device.  Its scratch (candidate lists, per-row counters)
+ * is one static 8 MiB device array that every GPU loading the library holds
+ * until the process exits; rows x ceil(N / chunk) x K candidate entries must
+ * fit in it (about 1M entries), else IDX_ENOWORKSPACE.  The call allocates
+ * nothing: the first call on a device looks up the array's device address
+ * (do that first call before any stream capture), and every call clears the
+ * counters it uses with cudaMemsetAsync on `stream`.  All calls share the
+ * array, which keeps the last call's contents, so calls that overlap on the
+ * GPU race; clamped lengths are not reported (there is no status to read).
+ */
+IDX_API int topk_select_noalloc(const float* scores, const int32_t* lengths, int rows, int N,
+                                int64_t lds, int K, int32_t* idx_out, float* val_out,
+                                idx_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

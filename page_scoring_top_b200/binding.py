@@ -35,6 +35,7 @@ SIGNATURES = {
     "idx_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "idx_strerror": (ctypes.c_char_p, [_I]),
     "idx_num_sms": (_I, [_P]),
+    "topk_select_noalloc": (_I, [_P, _P, _I, _I, _L, _I, _P, _P, _P]),
 }
 
 _lib = None
@@ -156,6 +157,17 @@ def topk_select(ctx, scores, lengths, K, idx_out, val_out=None, stream=None):
     _check(lib().topk_select(ctx.handle, _ptr(scores), _ptr(lengths), rows, N, scores.stride(0), K,
                              _ptr(idx_out), _ptr(val_out), _stream(stream, scores.device)),
            "topk_select")
+    return idx_out, val_out
+
+
+def topk_select_noalloc(scores, lengths, K, idx_out, val_out=None, stream=None):
+    """topk_select without a context: scratch in a static device array (see idx.h)."""
+    if scores.dim() != 2 or scores.stride(1) != 1:
+        raise ValueError("scores must be 2-D with unit column stride")
+    rows, N = scores.shape
+    _check(lib().topk_select_noalloc(_ptr(scores), _ptr(lengths), rows, N, scores.stride(0), K,
+                                     _ptr(idx_out), _ptr(val_out), _stream(stream, scores.device)),
+           "topk_select_noalloc")
     return idx_out, val_out
 
 
