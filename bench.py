@@ -63,9 +63,10 @@ def dist_env():
 
 
 def workload_inputs(rank):
+    from page_scoring_top_b200 import dist as pdist
     from page_scoring_top_b200 import synth
     spec = dict(synth.WORKLOADS[WORKLOAD])
-    seed = spec["seed"] + 1000 * rank
+    seed = pdist.rank_seed(spec["seed"], rank)
     return synth.workload(WORKLOAD, seed=seed), spec, seed
 
 
@@ -272,14 +273,9 @@ def run_ours(args):
     clocks = sampler.stop()
     barrier()
     ms = ev0.elapsed_time(ev1)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    pages_t = torch.tensor([float(pages)], dtype=torch.float64, device=dev)
-    if pg is not None:
-        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
-        pg.all_reduce(pages_t, op=pg.ReduceOp.SUM)
-    ms_max = float(ms_t.item())
+    from page_scoring_top_b200 import dist as pdist
+    ms_max, total_pages = pdist.reduce_timing(ms, pages, device=dev)
     ms_per_step = ms_max / args.steps
-    total_pages = float(pages_t.item())
     value = total_pages * args.steps / (ms_max * 1e-3)
     rc, bits = binding.idx_get_status(ctx)
     if rc != 0:
@@ -371,14 +367,11 @@ def measure_e2e(binding, ctx, d, K, dev, stream, steps, barrier, pg):
     torch.cuda.synchronize(dev)
     barrier()
     ms = e0.elapsed_time(e1)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    pages_t = torch.tensor([float(sum(lengths))], dtype=torch.float64, device=dev)
-    if pg is not None:
-        pg.all_reduce(ms_t, op=pg.ReduceOp.MAX)
-        pg.all_reduce(pages_t, op=pg.ReduceOp.SUM)
-    value = float(pages_t.item()) * steps / (float(ms_t.item()) * 1e-3)
+    from page_scoring_top_b200 import dist as pdist
+    ms_max, total_pages = pdist.reduce_timing(ms, sum(lengths), device=dev)
+    value = total_pages * steps / (ms_max * 1e-3)
     return {"value": value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": steps, "ms_per_step": float(ms_t.item()) / steps}
+            "steps": steps, "ms_per_step": ms_max / steps}
 
 
 def main():
