@@ -39,7 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per valid page of the fused decode kernel, from the ncu capture
 # summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum per
 # launch / pages per launch); None until a capture of the current kernel exists.
-NCU_TRAFFIC_BYTES_PER_PAGE = None
+NCU_TRAFFIC_BYTES_PER_PAGE = None  # the kernel changed after the last capture
 
 
 def parse():
@@ -312,7 +312,7 @@ def run_ours(args):
             "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "kernel": "decode_kernel<16,1,fused>"},
+                         "kernel": "decode_kernel<128,1,fused>"},
             "gpu_launches": args.steps,
             "clocks": clocks,
             "e2e": e2e,
