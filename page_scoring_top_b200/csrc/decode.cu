@@ -33,23 +33,23 @@
 // bit-identical.
 #include "common.cuh"
 #include "kernels.h"
-#include "select.cuh"
+#include "fused.cuh"
 
 namespace idx {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = kConsumerWarps * 32;
+static_assert(kConsumers == kSelThreads, "the consumer warps run the select steps");
 constexpr int kDecodeThreads = kConsumers + 32;
 constexpr int kStagePages = 32;
 constexpr int kMaxStages = 32;
 constexpr int kLMin = 256;
 constexpr int kSmemMax = 227 * 1024;
-constexpr int kMaxFusedT = 4;
 constexpr int kProducerLanes = 4;
 constexpr size_t kRingTargetBytes = 128 * 1024;
 
 struct DecodeLayout {
-  size_t ring, fbuf, fstate, scratch, sortv, sortb, off, bar, misc, total;
+  size_t ring, fbuf, fstate, scratch, sortv, sortb, hist, off, bar, misc, total;
   int nstage;
   int cap;  // filter entries per token
 };
@@ -60,9 +60,7 @@ __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~(size_t
 __host__ __device__ inline DecodeLayout decode_layout(bool fused, int D, int T) {
   DecodeLayout L;
   const size_t stage_bytes = (size_t)kStagePages * D * 2;
-  int tp = 1;
-  while (tp < T) tp <<= 1;
-  L.cap = fused ? kFilterCap / tp : 0;
+  L.cap = fused ? fused_cap(T) : 0;
   size_t o = 0;
   L.fbuf = o;  // per token: cap bits then cap indices; 2 * kFilterCap words in all
   o += fused ? (size_t)kFilterCap * 8 : 0;
@@ -74,6 +72,8 @@ __host__ __device__ inline DecodeLayout decode_layout(bool fused, int D, int T) 
   o += fused ? (size_t)(kMaxK + 2) * 8 : 0;
   L.sortb = o;
   o += fused ? (size_t)(kMaxK + 4) * 4 : 0;
+  L.hist = o;  // single-token filters also keep their digit histograms
+  o += (fused && T == 1) ? (size_t)(kHBins + kHCoarse) * 4 : 0;
   L.off = o;
   o += align16((size_t)(kDecodeMaxB + 1) * 4);
   L.bar = o;
@@ -98,29 +98,6 @@ __host__ __device__ inline DecodeLayout decode_layout(bool fused, int D, int T) 
   return L;
 }
 
-// First request b whose pages extend past global page gp (s_off[b+1] > gp).
-__device__ __forceinline__ int row_of(const int* s_off, int B, int gp) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (s_off[mid + 1] > gp) hi = mid;
-    else lo = mid + 1;
-  }
-  return lo;
-}
-
-// Local page index in request b of the chunk boundary at global page x, snapped
-// down to a multiple of the stage size (or clamped to the row's ends).  Every
-// stage then starts at a request-local page index that is a multiple of 32, so
-// the arithmetic order of a page's score depends on the page alone, not on how
-// the batch was cut into chunks.
-__device__ __forceinline__ int snap_local(const int* s_off, int b, int x) {
-  const int len = s_off[b + 1] - s_off[b];
-  const int r = x - s_off[b];
-  if (r >= len) return len;
-  return r <= 0 ? 0 : (r & ~(kStagePages - 1));
-}
-
 // Unpack 8 bf16 (one 16-byte chunk) to fp32; element 2k is the low half of word k.
 __device__ __forceinline__ void unpack8(const uint4 v, float* f) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -135,6 +112,9 @@ __device__ __forceinline__ void unpack8(const uint4 v, float* f) {
 template <int D_T, int TT, bool FUSED>
 __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
+  // One token per row: its filter keeps a digit histogram (hsel.cuh), which
+  // supplies the running threshold, the winners and the output order.
+  constexpr bool HIST = FUSED && TT == 1;
   constexpr int CPL = D_T ? D_T / 32 : 8;  // 16-byte chunks per lane (max)
   const int D = D_T ? D_T : a.D;
   const DecodeLayout L = decode_layout(FUSED, D, a.T);
@@ -144,13 +124,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   SelectScratch& sc = *reinterpret_cast<SelectScratch*>(smem + L.scratch);
   uint64_t* sortv = reinterpret_cast<uint64_t*>(smem + L.sortv);
   uint32_t* sortb = reinterpret_cast<uint32_t*>(smem + L.sortb);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);
   int* s_off = reinterpret_cast<int*>(smem + L.off);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* empty = full + kMaxStages;
   int* misc = reinterpret_cast<int*>(smem + L.misc);
   volatile int* s_abort = misc;
-  int* s_flag = misc + 1;
   uint32_t* s_wsum = reinterpret_cast<uint32_t*>(misc + 4);  // 9 warp sums
+  const FusedSel fsel{fbuf, fst, &sc, sortv, sortb, hist, L.cap, misc + 1};
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -171,33 +152,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
     *s_abort = 0;
     fence_mbar_init();
   }
-  // Prefix sums of the clamped lengths: s_off[b] = first global page of request b.
-  {
-    int running = 0;
-    if (tid == 0) s_off[0] = 0;
-    for (int base = 0; base < B; base += kDecodeThreads) {
-      const int i = base + tid;
-      int len = 0;
-      if (i < B) {
-        len = a.lengths ? a.lengths[i] : N;
-        if (len < 0 || len > N) {
-          if (g == 0) atomicOr(a.status, kErrLengthClamped);
-          len = len < 0 ? 0 : N;
-        }
-      }
-      const uint32_t incl = warp_incl_scan((uint32_t)len);
-      if (lane == 31) s_wsum[warp] = incl;
-      __syncthreads();
-      uint32_t excl = incl - (uint32_t)len, total = 0;
-      for (int w = 0; w < kDecodeThreads / 32; ++w) {
-        if (w < warp) excl += s_wsum[w];
-        total += s_wsum[w];
-      }
-      if (i < B) s_off[i + 1] = running + (int)excl + len;
-      __syncthreads();
-      running += (int)total;
-    }
-  }
+  length_prefix(a, s_off, s_wsum, kDecodeThreads);
   __syncthreads();
   const int P = s_off[B];
   int Lc = (P + G - 1) / G;
@@ -246,32 +201,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   }
 
   // ------------------------------------------------------------------ consumers
-  if (!FUSED) {
-    // -inf for the padded pages p >= len[b] of every token row: rows are cut
-    // into 4096-entry pieces dealt round-robin to the CTAs.
-    constexpr int kPiece = 4096;
-    const int ppr = (N + kPiece - 1) / kPiece;  // pieces per row
-    const int64_t npieces = (int64_t)B * T * ppr;
-    for (int64_t pc = g; pc < npieces; pc += G) {
-      const int rowi = (int)(pc / ppr);
-      const int b = rowi / T;
-      const int lb = s_off[b + 1] - s_off[b];
-      const int p_lo = max(lb, (int)(pc - (int64_t)rowi * ppr) * kPiece);
-      const int p_hi = min(N, (int)(pc - (int64_t)rowi * ppr) * kPiece + kPiece);
-      float* dst = a.scores + (int64_t)rowi * N;
-      for (int p = p_lo + tid; p < p_hi; p += kConsumers) dst[p] = __uint_as_float(kNegInfBits);
-    }
-  } else {
-    // Rows with no valid page: their output is all padding.
-    for (int b = g; b < B; b += G) {
-      if (s_off[b + 1] != s_off[b]) continue;
-      for (int x = tid; x < T * a.K; x += kConsumers) {
-        const int64_t o = ((int64_t)b * T) * a.K + x;
-        a.idx_out[o] = -1;
-        if (a.val_out) a.val_out[o] = __uint_as_float(kNegInfBits);
-      }
-    }
-  }
+  if (!FUSED) score_padding(a, s_off, g, G);
+  else fused_empty_rows(a, s_off, g, G);
 
   // Lane geometry: lane = 4 * pg + c4; page-group pg (0..7) of each 8-page
   // instruction, lane c4 (0..3) within the page.
@@ -290,12 +221,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
     lane_off[jj] = (uint32_t)pg * page_bytes + (uint32_t)ch * 16u;
   }
   const int my_page = c4 * 8 + pg;  // page this lane holds after the butterfly
-  // Check the filters every `rounds` rounds of 8 stages (a round appends at
-  // most 256 entries per token), and compact a token's filter once it holds a
-  // few K entries (early, so the threshold rises fast) and always before the
-  // next check could overflow it.
-  const int rounds = FUSED ? max(1, min(4, (cap - a.K) / kConsumers)) : 1;
-  const int compact_at = min(cap - rounds * kConsumers, max(4 * a.K, 1024));
+  // Filter checks every `rounds` rounds of 8 stages (a round appends at most
+  // 256 entries per token).
+  const int rounds = FUSED ? fused_rounds(cap, a.K) : 1;
+  const int compact_at = FUSED ? fused_compact_at<HIST>(cap, a.K) : 0;
   const int check_period = rounds * kConsumerWarps;
   const bool q_resident = (T <= TT);
 
@@ -310,7 +239,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
       const int p0 = snap_local(s_off, b, cb);
       const int np = snap_local(s_off, b, ce) - p0;  // may be 0
       if (FUSED) {
-        if (tid < T) filter_reset(fst[tid]);
+        fused_begin<HIST>(fsel, T);
         group_sync(kConsumers);
       }
       for (int sp = 0; sp < np; sp += kStagePages, ++stage) {
@@ -383,9 +312,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
             for (int t = 0; t < TT; ++t) {
               if (t0 + t < T) {
                 if (FUSED) {
-                  uint32_t* fb = fbuf + (t0 + t) * 2 * cap;
-                  filter_offer(fst[t0 + t], fb, fb + cap, __float_as_uint(acc[t][0]),
-                               (uint32_t)(p0 + sp + my_page), mine);
+                  fused_offer<HIST>(fsel, t0 + t, __float_as_uint(acc[t][0]),
+                                    (uint32_t)(p0 + sp + my_page), mine);
                 } else if (mine) {
                   a.scores[((int64_t)b * T + t0 + t) * N + p0 + sp + my_page] = acc[t][0];
                 }
@@ -394,46 +322,17 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&empty[slot]);
+          // Every fourth of its stages, a warp lifts the threshold to the
+          // histogram's top-K bin; two warps of each round do it.
+          if (HIST && ((stage >> 3) & 3) == (uint32_t)(warp & 3)) fused_raise(fsel, a.K);
         }
         if (FUSED && ((stage % check_period) == check_period - 1 || sp + kStagePages >= np)) {
           group_sync(kConsumers);  // this round's offers are complete
-          for (int t = 0; t < T; ++t)
-            if (fst[t].count > compact_at)
-              filter_compact<kConsumers>(fst[t], fbuf + t * 2 * cap, fbuf + t * 2 * cap + cap,
-                                         a.K, sc);
+          fused_check<HIST>(fsel, T, a.K, compact_at);
         }
       }
-      if (FUSED) {
-        const int j0 = s_off[b] / Lc;
-        const int j1 = (s_off[b + 1] - 1) / Lc;
-        for (int t = 0; t < T; ++t) {
-          uint32_t* fb = fbuf + t * 2 * cap;
-          uint32_t* fi = fb + cap;
-          filter_compact<kConsumers>(fst[t], fb, fi, a.K, sc);
-          const int kk = fst[t].count;
-          const int64_t orow = (int64_t)b * T + t;
-          if (j0 == j1) {
-            sort_and_write<kConsumers>(fb, fi, kk, a.K, sortv, sortb, a.idx_out + orow * a.K,
-                                       a.val_out ? a.val_out + orow * a.K : nullptr);
-          } else {
-            const int64_t slot = (int64_t)(j + b) * T + t;
-            publish_candidates<kConsumers>(fb, fi, kk, a.K, fst[t].thr,
-                                           a.cand_bits + slot * a.slot_stride,
-                                           a.cand_idx + slot * a.slot_stride, a.row_thr + orow);
-          }
-        }
-        if (j0 != j1 && arrive_last<kConsumers>(a.arrive + b, j1 - j0 + 1, s_flag)) {
-          for (int t = 0; t < T; ++t) {
-            const int64_t orow = (int64_t)b * T + t;
-            merge_candidates<kConsumers>(
-                j1 - j0 + 1, [=](int i) { return (int64_t)(j0 + i + b) * T + t; }, a.cand_bits,
-                a.cand_idx, a.slot_stride, a.K, a.row_thr + orow, fst[0], fbuf,
-                fbuf + kFilterCap, kFilterCap, sc, sortv, sortb, a.idx_out + orow * a.K,
-                a.val_out ? a.val_out + orow * a.K : nullptr);
-          }
-        }
-        group_sync(kConsumers);
-      }
+      if (FUSED)
+        fused_finalize<HIST>(fsel, a, T, b, j, s_off[b] / Lc, (s_off[b + 1] - 1) / Lc);
     }
   }
 }
@@ -473,6 +372,10 @@ static cudaError_t launch_tt(const DecodeArgs& a, int grid, cudaStream_t stream)
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream) {
+  // Head dims 64 and 128 with up to 64 query rows take the tensor-core kernel
+  // (decode_tc.cu), in both modes so that fused and score-mode scores stay
+  // bit-identical; the CUDA-core kernel takes every other shape.
+  if (decode_tc_supported(a.T, a.Q, a.D, a.ldc_b, a.c)) return launch_decode_tc(a, fused, num_sms, stream);
   const int grid = decode_grid(num_sms);
   if (fused) {
     if (a.D == 128) return launch_tt<128, true>(a, grid, stream);

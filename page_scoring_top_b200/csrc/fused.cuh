@@ -1,0 +1,237 @@
+// fused.cuh -- the select side of the fused score + top-K kernels.
+//
+// A decode kernel cuts the valid pages of a batch into one chunk per CTA; a
+// chunk covers the tail of one request, whole requests, the head of another.
+// Each (chunk, request) piece is a segment.  Per segment and token the kernel
+// feeds every page score to an exact online filter (select.cuh; with one
+// token per row the filter also keeps its digit histogram, hsel.cuh) and at
+// the segment's end either writes the row (the request lies inside the chunk)
+// or publishes the segment's top K to a candidate slot; the last CTA to
+// publish for a request merges the slots into the final row.  Top-K
+// selection ("Iterate Topk", opening description) over the page scores of
+// "Iterate Centroids Score"; the tie rule of "Round 18 Track C", section 2.
+#pragma once
+
+#include "hsel.cuh"
+#include "kernels.h"
+
+namespace idx {
+
+constexpr int kSelThreads = 256;  // threads 0..255 run every select step
+constexpr int kMaxFusedT = 4;
+
+// Shared-memory state of the fused select (pointers into the kernel's layout).
+struct FusedSel {
+  uint32_t* fbuf;       // per token: cap bits, then cap indices
+  FilterState* fst;     // per token
+  SelectScratch* sc;
+  uint64_t* sortv;      // kMaxK + 2 entries
+  uint32_t* sortb;      // kMaxK + 4 entries
+  uint32_t* hist;       // kHBins + kHCoarse words (single-token rows only)
+  int cap;              // filter entries per token
+  int* s_flag;
+};
+
+// Filter entries per token for T tokens.
+__host__ __device__ inline int fused_cap(int T) {
+  int tp = 1;
+  while (tp < T) tp <<= 1;
+  return kFilterCap / tp;
+}
+
+// Segment start (all select threads; the caller syncs after).
+template <bool HIST>
+__device__ __forceinline__ void fused_begin(const FusedSel& f, int T) {
+  if ((int)threadIdx.x < T) filter_reset(f.fst[threadIdx.x]);
+  if (HIST) hist_clear<kSelThreads>(f.hist, f.hist + kHBins);
+}
+
+// One warp offers its 32 lanes' scores of token t.
+template <bool HIST>
+__device__ __forceinline__ void fused_offer(const FusedSel& f, int t, uint32_t bits, uint32_t index,
+                                            bool valid) {
+  if (HIST) {
+    filter_offer_h(f.fst[0], f.fbuf, f.fbuf + f.cap, f.hist, f.hist + kHBins, bits, index, valid);
+  } else {
+    uint32_t* fb = f.fbuf + t * 2 * f.cap;
+    filter_offer(f.fst[t], fb, fb + f.cap, bits, index, valid);
+  }
+}
+
+// One warp lifts the single-token filter's threshold from its histogram.
+__device__ __forceinline__ void fused_raise(const FusedSel& f, int K) {
+  warp_raise_threshold(f.fst[0], f.hist, f.hist + kHBins, K);
+}
+
+// Overflow guard at a check point (all select threads, after a barrier that
+// completed every offer): compact a filter holding more than compact_at.
+template <bool HIST>
+__device__ __forceinline__ void fused_check(const FusedSel& f, int T, int K, int compact_at) {
+  for (int t = 0; t < T; ++t)
+    if (f.fst[t].count > compact_at) {
+      uint32_t* fb = f.fbuf + t * 2 * f.cap;
+      filter_compact<kSelThreads>(f.fst[t], fb, fb + f.cap, K, *f.sc);
+      if (HIST) hist_rebuild<kSelThreads>(f.fst[0], f.fbuf, f.fbuf + f.cap, f.hist, f.hist + kHBins);
+    }
+}
+
+// Check period (in rounds of 256 offers per token) and compaction mark: a
+// check comes before a filter could overflow; without a histogram the
+// compaction is also what raises the threshold, so it starts once a filter
+// holds a few K entries.
+__device__ __forceinline__ int fused_rounds(int cap, int K) {
+  return max(1, min(4, (cap - K) / kSelThreads));
+}
+template <bool HIST>
+__device__ __forceinline__ int fused_compact_at(int cap, int K) {
+  const int guard = cap - fused_rounds(cap, K) * kSelThreads;
+  return HIST ? guard : min(guard, max(4 * K, 1024));
+}
+
+// Segment end for request b, chunk j (all select threads, after a barrier
+// that completed every offer).  The request's pages span chunks j0..j1.
+template <bool HIST>
+__device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, int b, int j, int j0,
+                               int j1) {
+  SelectScratch& sc = *f.sc;
+  if (HIST) {
+    uint32_t* start = &sc.hist[0][0];  // kHBins words
+    const int kk = hist_winners<kSelThreads>(f.fst[0], f.fbuf, f.fbuf + f.cap, f.hist, a.K, sc,
+                                             f.sortv, f.sortb);
+    if (j0 == j1) {
+      hist_write_row<kSelThreads>(f.fbuf, f.fbuf + f.cap, kk, a.K, f.hist, start, sc, f.sortv,
+                                  f.sortb, a.idx_out + (int64_t)b * a.K,
+                                  a.val_out ? a.val_out + (int64_t)b * a.K : nullptr);
+    } else {
+      const int64_t slot = (int64_t)(j + b);
+      publish_candidates<kSelThreads>(f.fbuf, f.fbuf + f.cap, kk, a.K, f.fst[0].thr,
+                                      a.cand_bits + slot * a.slot_stride,
+                                      a.cand_idx + slot * a.slot_stride, a.row_thr + b);
+      if (arrive_last<kSelThreads>(a.arrive + b, j1 - j0 + 1, f.s_flag)) {
+        hist_merge<kSelThreads>(
+            j1 - j0 + 1, [=](int i) { return (int64_t)(j0 + i + b); }, a.cand_bits, a.cand_idx,
+            a.slot_stride, a.K, a.row_thr + b, f.fst[0], f.fbuf, f.fbuf + kFilterCap, kFilterCap,
+            f.hist, f.hist + kHBins, start, sc, f.sortv, f.sortb, a.idx_out + (int64_t)b * a.K,
+            a.val_out ? a.val_out + (int64_t)b * a.K : nullptr);
+      }
+    }
+  } else {
+    for (int t = 0; t < T; ++t) {
+      uint32_t* fb = f.fbuf + t * 2 * f.cap;
+      uint32_t* fi = fb + f.cap;
+      filter_compact<kSelThreads>(f.fst[t], fb, fi, a.K, sc);
+      const int kk = f.fst[t].count;
+      const int64_t orow = (int64_t)b * T + t;
+      if (j0 == j1) {
+        sort_and_write<kSelThreads>(fb, fi, kk, a.K, f.sortv, f.sortb, a.idx_out + orow * a.K,
+                                    a.val_out ? a.val_out + orow * a.K : nullptr);
+      } else {
+        const int64_t slot = (int64_t)(j + b) * T + t;
+        publish_candidates<kSelThreads>(fb, fi, kk, a.K, f.fst[t].thr,
+                                        a.cand_bits + slot * a.slot_stride,
+                                        a.cand_idx + slot * a.slot_stride, a.row_thr + orow);
+      }
+    }
+    if (j0 != j1 && arrive_last<kSelThreads>(a.arrive + b, j1 - j0 + 1, f.s_flag)) {
+      for (int t = 0; t < T; ++t) {
+        const int64_t orow = (int64_t)b * T + t;
+        merge_candidates<kSelThreads>(
+            j1 - j0 + 1, [=](int i) { return (int64_t)(j0 + i + b) * T + t; }, a.cand_bits,
+            a.cand_idx, a.slot_stride, a.K, a.row_thr + orow, f.fst[0], f.fbuf,
+            f.fbuf + kFilterCap, kFilterCap, sc, f.sortv, f.sortb, a.idx_out + orow * a.K,
+            a.val_out ? a.val_out + orow * a.K : nullptr);
+      }
+    }
+  }
+  group_sync(kSelThreads);
+}
+
+// Rows with no valid page get all-padding output (-1 / -inf), requests dealt
+// round-robin over the grid (all select threads).
+__device__ __forceinline__ void fused_empty_rows(const DecodeArgs& a, const int* s_off, int g,
+                                                 int G) {
+  for (int b = g; b < a.B; b += G) {
+    if (s_off[b + 1] != s_off[b]) continue;
+    for (int x = threadIdx.x; x < a.T * a.K; x += kSelThreads) {
+      const int64_t o = ((int64_t)b * a.T) * a.K + x;
+      a.idx_out[o] = -1;
+      if (a.val_out) a.val_out[o] = __uint_as_float(kNegInfBits);
+    }
+  }
+}
+
+// Score mode: -inf for the padded pages p >= len[b] of every token row; rows
+// are cut into 4096-entry pieces dealt round-robin over the grid.
+__device__ __forceinline__ void score_padding(const DecodeArgs& a, const int* s_off, int g, int G) {
+  constexpr int kPiece = 4096;
+  const int N = a.N, T = a.T;
+  const int ppr = (N + kPiece - 1) / kPiece;  // pieces per row
+  const int64_t npieces = (int64_t)a.B * T * ppr;
+  for (int64_t pc = g; pc < npieces; pc += G) {
+    const int rowi = (int)(pc / ppr);
+    const int b = rowi / T;
+    const int lb = s_off[b + 1] - s_off[b];
+    const int p_lo = max(lb, (int)(pc - (int64_t)rowi * ppr) * kPiece);
+    const int p_hi = min(N, (int)(pc - (int64_t)rowi * ppr) * kPiece + kPiece);
+    float* dst = a.scores + (int64_t)rowi * N;
+    for (int p = p_lo + (int)threadIdx.x; p < p_hi; p += kSelThreads)
+      dst[p] = __uint_as_float(kNegInfBits);
+  }
+}
+
+// Prefix sums of the clamped request lengths: s_off[b] = first global page of
+// request b, s_off[B] = all valid pages (all nthreads threads; s_wsum holds
+// one word per warp).  A length outside [0, N] is clamped and reported.
+__device__ __forceinline__ void length_prefix(const DecodeArgs& a, int* s_off, uint32_t* s_wsum,
+                                              int nthreads) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int running = 0;
+  if (tid == 0) s_off[0] = 0;
+  for (int base = 0; base < a.B; base += nthreads) {
+    const int i = base + tid;
+    int len = 0;
+    if (i < a.B) {
+      len = a.lengths ? a.lengths[i] : a.N;
+      if (len < 0 || len > a.N) {
+        if (blockIdx.x == 0) atomicOr(a.status, kErrLengthClamped);
+        len = len < 0 ? 0 : a.N;
+      }
+    }
+    const uint32_t incl = warp_incl_scan((uint32_t)len);
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    uint32_t excl = incl - (uint32_t)len, total = 0;
+    for (int w = 0; w < nthreads / 32; ++w) {
+      if (w < warp) excl += s_wsum[w];
+      total += s_wsum[w];
+    }
+    if (i < a.B) s_off[i + 1] = running + (int)excl + len;
+    __syncthreads();
+    running += (int)total;
+  }
+}
+
+// First request b whose pages extend past global page gp (s_off[b+1] > gp).
+__device__ __forceinline__ int row_of(const int* s_off, int B, int gp) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (s_off[mid + 1] > gp) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Local page index in request b of the chunk boundary at global page x, snapped
+// down to a multiple of 32 pages (or clamped to the row's ends).  Every
+// segment then starts at a request-local page index that is a multiple of 32,
+// so the arithmetic of a page's score depends on the page alone, not on how
+// the batch was cut into chunks.
+__device__ __forceinline__ int snap_local(const int* s_off, int b, int x) {
+  const int len = s_off[b + 1] - s_off[b];
+  const int r = x - s_off[b];
+  if (r >= len) return len;
+  return r <= 0 ? 0 : (r & ~31);
+}
+
+}  // namespace idx

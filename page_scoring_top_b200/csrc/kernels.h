@@ -57,6 +57,10 @@ int64_t decode_fused_slots(int64_t B, int64_t T, int64_t N, int grid);
 int decode_fused_max_k(int T);
 int decode_grid(int num_sms);
 cudaError_t launch_decode(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream);
+// Tensor-core decode kernel (decode_tc.cu): D in {64, 128}, T*Q <= 64,
+// 16-byte aligned request rows.  launch_decode routes these shapes to it.
+bool decode_tc_supported(int T, int Q, int D, int64_t ldc_b, const void* c);
+cudaError_t launch_decode_tc(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- prefill (tcgen05) score
 struct PrefillArgs {

@@ -29,6 +29,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace idx {
 
@@ -56,82 +57,12 @@ struct PfSmem {
   static_assert(tiles + (kPfMaxB + 1) * 4 <= a, "small state overflows");
 };
 
+constexpr uint32_t kPfIdesc = umma_idesc_bf16(kPfM, kPfTileN);
+
 struct PfParams {
   PrefillArgs a;
   int rows_per_req;  // T * Q
 };
-
-// ---------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                           uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
-                                           uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// K-major, 128-byte-swizzled operand: rows of 128 B, 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);          // start address
-  d |= (uint64_t)1u << 16;                          // leading byte offset (unused, 16 B)
-  d |= (uint64_t)(1024u >> 4) << 32;                // stride byte offset: 8 rows x 128 B
-  d |= (uint64_t)1u << 46;                          // descriptor version (sm_100)
-  d |= (uint64_t)2u << 61;                          // layout: SWIZZLE_128B
-  return d;
-}
-
-// kind::f16 instruction descriptor: BF16 x BF16 -> F32, K-major A and B.
-constexpr uint32_t kPfIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kPfTileN >> 3) << 17) |
-                              ((uint32_t)(kPfM >> 4) << 24);
-
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(kPfIdesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-      "%30, %31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 // Tile t of this CTA's sequence -> (request, first page).  s_tiles[b] is the
 // number of 256-page tiles before request b.
@@ -296,7 +227,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const uint32_t kb = (uint32_t)(k >> 2), ks = (uint32_t)(k & 3);
           const uint64_t ad = umma_desc_sw128(a_base + kb * kPfBlockA + ks * 32u);
           const uint64_t bd = umma_desc_sw128(b_base + kb * kPfBlockB + ks * 32u);
-          umma_bf16(d_tmem, ad, bd, k > 0 ? 1u : 0u);
+          umma_bf16(d_tmem, ad, bd, kPfIdesc, k > 0 ? 1u : 0u);
         }
         umma_commit(&empty[s]);
         umma_commit(&acc_full[acc]);
@@ -372,7 +303,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* p = nullptr;

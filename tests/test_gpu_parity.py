@@ -232,3 +232,56 @@ def test_length_out_of_range_is_clamped_and_reported(ctx):
     assert np.array_equal(got[0], ref_idx[0])        # 400 clamped to N = 300
     assert np.all(got[1] == -1)                      # -5 clamped to 0 pages
     _status_clean(ctx)
+
+
+# ------------------------------------------------------------------ fused select, adversarial orders
+
+def _ordered_inputs(order, B, N, lengths, seed):
+    """Inputs whose scores are set by two centroid coordinates: q puts 1 on
+    dim 0 and 2^-8 on dim 1 of head 0 (zeros elsewhere), so every score is
+    c[p,0] + c[p,1] / 256 exactly in fp32.  Orders:
+    ascending / descending: strictly monotone scores along the row (each page
+        beats every earlier one, or none), the worst and best visiting orders
+        of an online filter;
+    one_bin: all scores in [1, 1 + 1/256): one 12-bit digit bin, ~128 distinct
+        values, so the boundary bin is crowded and ties are everywhere;
+    few_values: scores in {-1, 0, 1, 2}."""
+    d = synth.decode_inputs(seed, B=B, T=1, Q=4, D=128, N=N, lengths=lengths)
+    q = np.zeros_like(d["q"])
+    q[:, :, 0, 0] = 0x3F80          # 1.0
+    q[:, :, 0, 1] = 0x3B80          # 2^-8
+    d["q"] = q
+    rng = np.random.default_rng(seed)
+    c = d["c"]
+    for b in range(B):
+        n = int(lengths[b])
+        c[b, :n, :] = 0
+        p = np.arange(n)
+        if order == "ascending":
+            c[b, :n, 0] = 0x3F80 + (p % 16000)      # bf16 patterns, increasing
+            c[b, :n, 1] = 0
+        elif order == "descending":
+            c[b, :n, 0] = 0x3F80 + ((n - 1 - p) % 16000)
+        elif order == "one_bin":
+            c[b, :n, 0] = 0x3F80
+            c[b, :n, 1] = 0x3F00 + rng.integers(0, 128, n)  # bf16 in [0.5, 1)
+        else:
+            c[b, :n, 0] = np.array([0xBF80, 0x0000, 0x3F80, 0x4000], np.uint16)[
+                rng.integers(0, 4, n)]
+    return d
+
+
+@pytest.mark.parametrize("order", ["ascending", "descending", "one_bin", "few_values"])
+@pytest.mark.parametrize("K", [256, 1000])
+def test_fused_adversarial_orders_long_rows(ctx, order, K):
+    lengths = np.array([16000, 15001], np.int32)
+    d = _ordered_inputs(order, 2, 16000, lengths, 610)
+    check_indexer(ctx, d, K=K)
+
+
+@pytest.mark.parametrize("order", ["ascending", "one_bin", "few_values"])
+def test_fused_adversarial_orders_short_rows(ctx, order):
+    rng = np.random.default_rng(611)
+    lengths = rng.integers(1, 3000, 64).astype(np.int32)
+    d = _ordered_inputs(order, 64, 3000, lengths, 612)
+    check_indexer(ctx, d, K=300)
