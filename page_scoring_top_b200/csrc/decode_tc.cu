@@ -349,8 +349,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
               }
             }
-            // one warp per tile lifts the threshold from the histogram
-            if (HIST && (int)((tile >> 1) & 3) == quad) fused_raise(fsel, a.K);
+            // every other tile, one warp lifts the threshold from the histogram
+            if (HIST && (int)((tile >> 1) & 7) == quad) fused_raise(fsel, a.K);
           }
           if (FUSED && ((tt + 1) % check_tiles == 0 || tt + 1 == ntl)) {
             group_sync(kTcEpi);  // every offer so far is complete

@@ -58,9 +58,10 @@ __device__ __forceinline__ void fused_offer(const FusedSel& f, int t, uint32_t b
   }
 }
 
-// One warp lifts the single-token filter's threshold from its histogram.
+// Lane 0 of the calling warp lifts the single-token filter's threshold from
+// its histogram.
 __device__ __forceinline__ void fused_raise(const FusedSel& f, int K) {
-  warp_raise_threshold(f.fst[0], f.hist, f.hist + kHBins, K);
+  if (lane_id() == 0) raise_threshold_1t(f.fst[0], f.hist, f.hist + kHBins, K);
 }
 
 // Overflow guard at a check point (all select threads, after a barrier that
@@ -95,25 +96,55 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
                                int j1) {
   SelectScratch& sc = *f.sc;
   if (HIST) {
+    // One token per row: the filter histogram is exact for the buffer, so one
+    // scan finds the boundary bin and the winners are placed from registers.
+    FilterState& fs = f.fst[0];
+    uint32_t* fb = f.fbuf;
+    uint32_t* fi = f.fbuf + f.cap;
     uint32_t* start = &sc.hist[0][0];  // kHBins words
-    const int kk = hist_winners<kSelThreads>(f.fst[0], f.fbuf, f.fbuf + f.cap, f.hist, a.K, sc,
-                                             f.sortv, f.sortb);
-    if (j0 == j1) {
-      hist_write_row<kSelThreads>(f.fbuf, f.fbuf + f.cap, kk, a.K, f.hist, start, sc, f.sortv,
-                                  f.sortb, a.idx_out + (int64_t)b * a.K,
-                                  a.val_out ? a.val_out + (int64_t)b * a.K : nullptr);
-    } else {
-      const int64_t slot = (int64_t)(j + b);
-      publish_candidates<kSelThreads>(f.fbuf, f.fbuf + f.cap, kk, a.K, f.fst[0].thr,
+    // boundary-bin members go to the front of the buffer once it is in registers
+    uint64_t* bl_v = reinterpret_cast<uint64_t*>(f.fbuf);
+    uint32_t* bl_b = f.fbuf + 2 * (kBoundaryMax + 2);
+    const bool single = j0 == j1;
+    int32_t* out_i = a.idx_out + (int64_t)b * a.K;
+    float* out_v = a.val_out ? a.val_out + (int64_t)b * a.K : nullptr;
+    const int64_t slot = (int64_t)(j + b);
+    hist_scan<kSelThreads>(f.hist, start, (uint32_t)a.K, sc);
+    if (sc.bcast[0] == 0xFFFFFFFFu || sc.bcast[2] <= (uint32_t)kBoundaryMax) {
+      constexpr int E = kFilterCap / kSelThreads;
+      uint64_t v[E];
+      uint32_t bits[E];
+      const int nk = load_buffer<kSelThreads, E>(fb, fi, fs.count, v, bits);
+      group_sync(kSelThreads);
+      if (single)
+        place_ordered<kSelThreads, E>(v, bits, nk, f.hist, start, a.K, sc, f.sortv, f.sortb, bl_v,
+                                      bl_b, out_i, out_v);
+      else
+        place_publish<kSelThreads, E>(v, bits, nk, start, a.K, sc, bl_v, bl_b,
                                       a.cand_bits + slot * a.slot_stride,
                                       a.cand_idx + slot * a.slot_stride, a.row_thr + b);
-      if (arrive_last<kSelThreads>(a.arrive + b, j1 - j0 + 1, f.s_flag)) {
-        hist_merge<kSelThreads>(
-            j1 - j0 + 1, [=](int i) { return (int64_t)(j0 + i + b); }, a.cand_bits, a.cand_idx,
-            a.slot_stride, a.K, a.row_thr + b, f.fst[0], f.fbuf, f.fbuf + kFilterCap, kFilterCap,
-            f.hist, f.hist + kHBins, start, sc, f.sortv, f.sortb, a.idx_out + (int64_t)b * a.K,
-            a.val_out ? a.val_out + (int64_t)b * a.K : nullptr);
-      }
+    } else {
+      // a crowded boundary bin (heavy ties): radix compaction, then a plain write
+      filter_compact<kSelThreads>(fs, fb, fi, a.K, sc);
+      if (single)
+        sort_and_write<kSelThreads>(fb, fi, fs.count, a.K, f.sortv, f.sortb, out_i, out_v);
+      else
+        publish_candidates<kSelThreads>(fb, fi, fs.count, a.K, fs.thr,
+                                        a.cand_bits + slot * a.slot_stride,
+                                        a.cand_idx + slot * a.slot_stride, a.row_thr + b);
+    }
+    if (!single && arrive_last<kSelThreads>(a.arrive + b, j1 - j0 + 1, f.s_flag)) {
+      const int nslots = j1 - j0 + 1;
+      auto slot_of = [=](int i) { return (int64_t)(j0 + i + b); };
+      bool done = false;
+      if (nslots * a.K <= kFilterCap)
+        done = hist_merge_regs<kSelThreads, kFilterCap / kSelThreads>(
+            nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride, a.K, a.row_thr + b, f.hist,
+            start, sc, f.sortv, f.sortb, bl_v, bl_b, out_i, out_v);
+      if (!done)
+        merge_candidates<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride,
+                                      a.K, a.row_thr + b, fs, f.fbuf, f.fbuf + kFilterCap,
+                                      kFilterCap, sc, f.sortv, f.sortb, out_i, out_v);
     }
   } else {
     for (int t = 0; t < T; ++t) {

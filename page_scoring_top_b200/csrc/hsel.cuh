@@ -33,33 +33,27 @@ constexpr int kHBins = 1 << kHBits;          // 4096 fine bins
 constexpr int kHShift = 32 - kHBits;         // digit = key >> kHShift
 constexpr int kHCoarse = kHBins / 32;        // 128 coarse bins of 32 fine bins
 constexpr int kBoundaryMax = 256;            // bin-b members resolved by counting
-constexpr int kSortBinMax = 128;             // largest bin ordered by counting
 
 __device__ __forceinline__ uint32_t hdigit_v(uint64_t v) {
   return (uint32_t)(v >> (32 + kHShift));
 }
 
 // filter_offer that also counts every appended entry in the fine and coarse
-// histograms of the buffer (hist: kHBins words, chist: kHCoarse words).
+// histograms of the buffer (hist: kHBins words, chist: kHCoarse words).  Each
+// taking lane claims its slot with its own shared-memory atomic: after the
+// first few hundred offers only a few lanes of a warp take, and a ballot and
+// shuffle per warp cost more than those atomics.
 __device__ __forceinline__ void filter_offer_h(FilterState& fs, uint32_t* fb, uint32_t* fi,
                                                uint32_t* hist, uint32_t* chist, uint32_t bits,
                                                uint32_t index, bool valid) {
   const uint64_t v = valid ? rank_value(bits, index) : 0ull;
-  const bool take = v > fs.thr;
-  const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
-  if (m) {
-    const int leader = __ffs(m) - 1;
-    int base = 0;
-    if ((int)lane_id() == leader) base = atomicAdd(&fs.count, __popc(m));
-    base = __shfl_sync(0xFFFFFFFFu, base, leader);
-    if (take) {
-      const int pos = base + __popc(m & lanemask_lt());
-      fb[pos] = bits;
-      fi[pos] = index;
-      const uint32_t d = hdigit_v(v);
-      atomicAdd(&hist[d], 1u);
-      atomicAdd(&chist[d >> 5], 1u);
-    }
+  if (v > fs.thr) {
+    const int pos = atomicAdd(&fs.count, 1);
+    fb[pos] = bits;
+    fi[pos] = index;
+    const uint32_t d = hdigit_v(v);
+    atomicAdd(&hist[d], 1u);
+    atomicAdd(&chist[d >> 5], 1u);
   }
 }
 
@@ -86,63 +80,64 @@ __device__ void hist_rebuild(const FilterState& fs, const uint32_t* fb, const ui
   group_sync(NT);
 }
 
-// One warp: the highest digit b >= 1 with at least K entries counted in bins
-// >= b, from a snapshot of histograms that other warps keep incrementing; 0
-// when fewer than K entries are counted.  Every count read is a lower bound
-// of the buffer's true count, so the answer is a valid lower bound of the
-// digit of the K-th largest buffered value.
-__device__ __forceinline__ uint32_t warp_hist_floor(const uint32_t* hist, const uint32_t* chist,
-                                                    uint32_t K) {
-  const int lane = (int)lane_id();
-  // coarse bins 127 - 4*lane - 3 .. 127 - 4*lane: lane 0 holds the top ones
-  const uint4 q = *reinterpret_cast<const uint4*>(chist + kHCoarse - 4 * (lane + 1));
-  const uint32_t s = q.x + q.y + q.z + q.w;
-  const uint32_t incl = warp_incl_scan(s);
-  const uint32_t m = __ballot_sync(0xFFFFFFFFu, incl >= K);
-  if (!m) return 0u;
-  const int L = __ffs(m) - 1;
-  uint32_t c = 0, above = 0;
-  if (lane == L) {
-    const uint32_t h[4] = {q.w, q.z, q.y, q.x};  // descending bins
-    uint32_t cum = incl - s;
-    bool found = false;
+// The highest digit b >= 1 with at least K entries counted in bins >= b, from
+// a snapshot of histograms that other warps keep incrementing; 0 when fewer
+// than K entries are counted.  Every count read is a lower bound of the
+// buffer's true count, so the answer is a valid lower bound of the digit of
+// the K-th largest buffered value.  One thread: coarse bins from the top
+// (16-byte loads) until K entries are reached, then the 32 fine bins of the
+// coarse bin that got there (no warp-synchronous steps: on this part a shuffle
+// or ballot in a loop costs more than a short scan by one lane).
+__device__ __forceinline__ uint32_t hist_floor_1t(const uint32_t* hist, const uint32_t* chist,
+                                                  uint32_t K) {
+  uint32_t cum = 0;
+  for (int c4 = kHCoarse / 4 - 1; c4 >= 0; --c4) {
+    const uint4 q = reinterpret_cast<const uint4*>(chist)[c4];
+    const uint32_t h[4] = {q.w, q.z, q.y, q.x};  // coarse bins 4*c4+3 .. 4*c4
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      if (!found && cum + h[k] >= K) {
-        c = (uint32_t)(kHCoarse - 1 - 4 * L - k);
-        above = cum;
-        found = true;
+      if (cum + h[k] >= K) {
+        const int c = 4 * c4 + 3 - k;
+        // fine bins of coarse bin c, top down; the coarse count alone
+        // already guarantees bin 32 * c
+        const uint4* f4 = reinterpret_cast<const uint4*>(hist + 32 * c);
+        for (int f = 7; f >= 0; --f) {
+          const uint4 w = f4[f];
+          const uint32_t g[4] = {w.w, w.z, w.y, w.x};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            cum += g[e];
+            if (cum >= K) return (uint32_t)(32 * c + 4 * f + 3 - e);
+          }
+        }
+        return (uint32_t)(32 * c);
       }
       cum += h[k];
     }
   }
-  c = __shfl_sync(0xFFFFFFFFu, c, L);
-  above = __shfl_sync(0xFFFFFFFFu, above, L);
-  // fine bins of coarse bin c, lane 0 the top one
-  const uint32_t f = hist[c * 32 + 31 - lane];
-  const uint32_t fincl = warp_incl_scan(f) + above;
-  const uint32_t m2 = __ballot_sync(0xFFFFFFFFu, fincl >= K);
-  // The coarse snapshot alone already guarantees bin c * 32.
-  return m2 ? c * 32 + 31 - (uint32_t)(__ffs(m2) - 1) : c * 32;
+  return 0u;
 }
 
-// Raise a filter's threshold to "digit >= b" (one warp, lane 0 writes).  A
-// racing raise by another warp may win with a lower value: that only admits
-// more entries.
-__device__ __forceinline__ void warp_raise_threshold(FilterState& fs, const uint32_t* hist,
-                                                     const uint32_t* chist, int K) {
-  const uint32_t b = warp_hist_floor(hist, chist, (uint32_t)K);
-  if (b != 0u && lane_id() == 0) {
+// Raise a filter's threshold to "digit >= b" (one thread).  A racing raise by
+// another warp may win with a lower value: that only admits more entries.
+__device__ __forceinline__ void raise_threshold_1t(FilterState& fs, const uint32_t* hist,
+                                                   const uint32_t* chist, int K) {
+  const uint32_t b = hist_floor_1t(hist, chist, (uint32_t)K);
+  if (b != 0u) {
     const unsigned long long t = ((unsigned long long)b << (32 + kHShift)) - 1ull;
     if (t > fs.thr) fs.thr = t;
   }
 }
 
-// Top-K boundary of an exact 4096-bin histogram (all NT threads).
-// Broadcasts: bcast[0] = b, bcast[1] = entries in bins above b, bcast[2] =
-// hist[b], bcast[3] = total; when total <= r only bcast[3] is meaningful.
+// Scan of an exact 4096-bin histogram (all NT threads, two barriers):
+// start[d] = entries in bins above d (exclusive suffix sum) and the top-K
+// boundary, broadcast as bcast[0] = b (the bin holding the K-th largest
+// entry; 0xFFFFFFFF when total <= K: every entry is a winner), bcast[1] =
+// entries above b, bcast[2] = hist[b], bcast[3] = total.  Each thread owns 16
+// consecutive bins (thread 0 the top ones), read and written 16 bytes at a time.
 template <int NT>
-__device__ __forceinline__ void hist_boundary(const uint32_t* hist, uint32_t r, SelectScratch& sc) {
+__device__ __forceinline__ void hist_scan(const uint32_t* hist, uint32_t* start, uint32_t K,
+                                          SelectScratch& sc) {
   constexpr int BPT = kHBins / NT;
   static_assert(kHBins % NT == 0 && BPT % 4 == 0, "bins per thread");
   const int tid = threadIdx.x;
@@ -170,259 +165,233 @@ __device__ __forceinline__ void hist_boundary(const uint32_t* hist, uint32_t r, 
     if (w < warp) excl += x;
     total += x;
   }
-  if (tid == 0) sc.bcast[3] = total;
-  if (total > r && excl < r && r <= excl + s) {
-    uint32_t cum = excl;
-    bool found = false;
-#pragma unroll
-    for (int k = BPT - 1; k >= 0; --k) {
-      if (!found && cum + h[k] >= r) {
-        sc.bcast[0] = (uint32_t)(lo + k);
-        sc.bcast[1] = cum;
-        sc.bcast[2] = h[k];
-        found = true;
-      }
-      cum += h[k];
+  if (tid == 0) {
+    sc.bcast[3] = total;
+    if (total <= K) {
+      sc.bcast[0] = 0xFFFFFFFFu;
+      sc.bcast[1] = total;
+      sc.bcast[2] = 0u;
     }
   }
+  uint32_t st[BPT];
+  uint32_t cum = excl;
+  bool found = !(total > K && excl < K && K <= excl + s);
+#pragma unroll
+  for (int k = BPT - 1; k >= 0; --k) {
+    st[k] = cum;
+    if (!found && cum + h[k] >= K) {
+      sc.bcast[0] = (uint32_t)(lo + k);
+      sc.bcast[1] = cum;
+      sc.bcast[2] = h[k];
+      found = true;
+    }
+    cum += h[k];
+  }
+#pragma unroll
+  for (int k = 0; k < BPT; k += 4)
+    *reinterpret_cast<uint4*>(start + lo + k) = make_uint4(st[k], st[k + 1], st[k + 2], st[k + 3]);
   group_sync(NT);
 }
 
-// Exact winners of a filter buffer whose histogram `hist` is exactly that of
-// its fs.count entries (and which holds the top K of everything offered).
-// Leaves the min(K, count) winners, unordered, at the front of fb/fi, sets
-// fs.count to their number and, when entries were dropped, fs.thr to the K-th
-// largest rank value (kept entries are >= it).  bl_v/bl_b: kBoundaryMax
-// entries of scratch.  All NT threads, after a barrier that completed every
-// offer; returns the winner count.
-template <int NT>
-__device__ int hist_winners(FilterState& fs, uint32_t* fb, uint32_t* fi, const uint32_t* hist,
-                            int K, SelectScratch& sc, uint64_t* bl_v, uint32_t* bl_b) {
-  constexpr int E = kFilterCap / NT;
-  const int tid = threadIdx.x;
-  hist_boundary<NT>(hist, (uint32_t)K, sc);
-  const int n = fs.count;
-  if (sc.bcast[3] <= (uint32_t)K) return n;  // everything buffered is a winner
-  const uint32_t b = sc.bcast[0];
-  const int above = (int)sc.bcast[1];
-  const int cnt = (int)sc.bcast[2];
-  const int r = K - above;
-  if (cnt > kBoundaryMax) {  // a crowded boundary bin (ties): radix compaction
-    filter_compact<NT>(fs, fb, fi, K, sc);
-    return fs.count;
-  }
-  const int nk = (n + NT - 1) / NT;
-  uint64_t v[E];
-  uint32_t bb[E];
-#pragma unroll
-  for (int k = 0; k < E; ++k) {
-    const int i = tid + k * NT;
-    v[k] = 0ull;
-    bb[k] = 0u;
-    if (k < nk && i < n) {
-      bb[k] = fb[i];
-      v[k] = rank_value(bb[k], fi[i]);
+// Rank each of the cnt members of the boundary bin (bl_v / bl_b; bl_v holds
+// a zero after the last member, 16-byte aligned) among the others and hand
+// the r largest to sink(rank, v, bits).  One member per thread, compared
+// against all members two at a time (rank values are unique).
+template <int NT, class Sink>
+__device__ __forceinline__ void rank_boundary(const uint64_t* bl_v, const uint32_t* bl_b, int cnt,
+                                              int r, Sink sink) {
+  const int half = (cnt + 1) >> 1;
+  for (int t = threadIdx.x; t < cnt; t += NT) {
+    const uint64_t x = bl_v[t];
+    int rank = 0;
+#pragma unroll 4
+    for (int j = 0; j < half; ++j) {
+      const ulonglong2 u = reinterpret_cast<const ulonglong2*>(bl_v)[j];
+      rank += (u.x > x) + (u.y > x);
     }
+    if (rank < r) sink(rank, x, bl_b[t]);
   }
-  if (tid == 0) {
-    sc.ctr = 0;
-    sc.pad[0] = 0;
-  }
-  group_sync(NT);  // every entry is in registers: the buffer front may be rewritten
-  const uint32_t lt = lanemask_lt();
+}
+
+// Split register-held entries (v[k], bits[k] for k < nk; v = 0 marks none)
+// by the boundary bin b of hist_scan, taking positions from the start[]
+// counters that hist_scan left: an entry of a higher bin calls win(v, bits,
+// digit, slot) with slot = start[digit]++ (so the winners fill [0, above),
+// grouped by bin, highest bin first); a member of bin b is appended to the
+// bl list at start[b]++ - above.
+template <int E, class Win>
+__device__ __forceinline__ void classify(const uint64_t (&v)[E], const uint32_t (&bits)[E], int nk,
+                                         uint32_t b, uint32_t above, uint32_t* start,
+                                         uint64_t* bl_v, uint32_t* bl_b, Win win) {
 #pragma unroll
   for (int k = 0; k < E; ++k) {
     if (k >= nk) break;
+    if (v[k] == 0) continue;
     const uint32_t d = hdigit_v(v[k]);
-    const bool win = v[k] != 0 && d > b;
-    const bool bnd = v[k] != 0 && d == b;
-    const uint32_t mw = __ballot_sync(0xFFFFFFFFu, win);
-    const uint32_t mb = __ballot_sync(0xFFFFFFFFu, bnd);
-    if (mw) {
-      const int leader = __ffs(mw) - 1;
-      int base = 0;
-      if ((int)lane_id() == leader) base = atomicAdd(&sc.ctr, __popc(mw));
-      base = __shfl_sync(0xFFFFFFFFu, base, leader);
-      if (win) {
-        const int pos = base + __popc(mw & lt);
-        fb[pos] = bb[k];
-        fi[pos] = ~(uint32_t)v[k];
-      }
-    }
-    if (mb) {
-      const int leader = __ffs(mb) - 1;
-      int base = 0;
-      if ((int)lane_id() == leader) base = atomicAdd(&sc.pad[0], __popc(mb));
-      base = __shfl_sync(0xFFFFFFFFu, base, leader);
-      if (bnd) {
-        const int pos = base + __popc(mb & lt);
-        bl_v[pos] = v[k];
-        bl_b[pos] = bb[k];
-      }
+    if (b == 0xFFFFFFFFu || d > b) {
+      win(v[k], bits[k], d, atomicAdd(&start[d], 1u));
+    } else if (d == b) {
+      const uint32_t p = atomicAdd(&start[d], 1u) - above;
+      bl_v[p] = v[k];
+      bl_b[p] = bits[k];
     }
   }
-  group_sync(NT);
-  // The r largest members of bin b follow the `above` sure winners; each
-  // member's place is the number of larger members (rank values are unique).
-  for (int t = tid; t < cnt; t += NT) {
-    const uint64_t x = bl_v[t];
-    int rank = 0;
-    for (int j = 0; j < cnt; ++j) rank += bl_v[j] > x;
-    if (rank < r) {
-      fb[above + rank] = bl_b[t];
-      fi[above + rank] = ~(uint32_t)x;
-      if (rank == r - 1) fs.thr = x;
-    }
-  }
-  if (tid == 0) fs.count = K;
-  group_sync(NT);
-  return K;
 }
 
-// Write the n (<= K) winners at the front of fb/fi as one output row in
-// descending order: position = winners in higher bins + rank among the
-// winners of the same bin.  cnt and start are kHBins-word scratch arrays
-// (cnt may alias the filter's histogram, which this overwrites); tv/tb hold
-// n entries.  A bin with more than kSortBinMax winners sends the row to
-// sort_and_write (tv/tb then need max(64, next_pow2(K)) + 1 entries).
-template <int NT>
-__device__ void hist_write_sorted(const uint32_t* fb, const uint32_t* fi, int n, int K,
-                                  uint32_t* cnt, uint32_t* start, SelectScratch& sc, uint64_t* tv,
-                                  uint32_t* tb, int32_t* idx_out, float* val_out) {
-  constexpr int BPT = kHBins / NT;
+// Exact top K of register-held entries, written as one ordered output row.
+// hist must be the exact histogram of the entries and hist_scan must have run
+// on it (start, sc.bcast) with no boundary bin above kBoundaryMax.  A
+// winner's position = winners in higher bins + its rank among the winners of
+// its bin; the r largest members of bin b follow all of them.  tv/tb stage
+// the winners (K entries); bl_v/bl_b hold kBoundaryMax + 2.  Slots past
+// min(K, total) get -1 / -inf.
+template <int NT, int E>
+__device__ void place_ordered(const uint64_t (&v)[E], const uint32_t (&bits)[E], int nk,
+                              const uint32_t* hist, uint32_t* start, int K, SelectScratch& sc,
+                              uint64_t* tv, uint32_t* tb, uint64_t* bl_v, uint32_t* bl_b,
+                              int32_t* idx_out, float* val_out) {
   const int tid = threadIdx.x;
-  for (int i = tid; i < kHBins; i += NT) cnt[i] = 0u;
-  if (tid == 0) sc.bcast[0] = 0u;
+  const uint32_t b = sc.bcast[0];
+  const int above = (int)sc.bcast[1];
+  const int cnt = (int)sc.bcast[2];
+  const int total = (int)sc.bcast[3];
+  classify(v, bits, nk, b, (uint32_t)above, start, bl_v, bl_b,
+           [&](uint64_t x, uint32_t xb, uint32_t, uint32_t slot) {
+             tv[slot] = x;
+             tb[slot] = xb;
+           });
+  if (tid == 0) bl_v[cnt] = 0ull;
   group_sync(NT);
-  for (int i = tid; i < n; i += NT) atomicAdd(&cnt[hdigit_v(rank_value(fb[i], fi[i]))], 1u);
-  group_sync(NT);
-  // exclusive suffix sums: start[d] = winners in bins above d
-  {
-    const int lo = kHBins - (tid + 1) * BPT;
-    uint32_t h[BPT];
-#pragma unroll
-    for (int k = 0; k < BPT; k += 4) {
-      const uint4 q = *reinterpret_cast<const uint4*>(cnt + lo + k);
-      h[k] = q.x;
-      h[k + 1] = q.y;
-      h[k + 2] = q.z;
-      h[k + 3] = q.w;
-    }
-    uint32_t s = 0, mx = 0;
-#pragma unroll
-    for (int k = 0; k < BPT; ++k) {
-      s += h[k];
-      mx = h[k] > mx ? h[k] : mx;
-    }
-    if (mx > (uint32_t)kSortBinMax) atomicMax(&sc.bcast[0], mx);
-    const uint32_t incl = warp_incl_scan(s);
-    const int warp = tid >> 5;
-    if (lane_id() == 31) sc.wsum[warp] = incl;
-    group_sync(NT);
-    if (sc.bcast[0] != 0u) {  // uniform: read after the barrier
-      sort_and_write<NT>(fb, fi, n, K, tv, tb, idx_out, val_out);
-      return;
-    }
-    uint32_t cum = incl - s;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w)
-      if (w < warp) cum += sc.wsum[w];
-#pragma unroll
-    for (int k = BPT - 1; k >= 0; --k) {
-      start[lo + k] = cum;
-      cum += h[k];
-    }
-  }
-  group_sync(NT);
-  for (int i = tid; i < n; i += NT) {
-    const uint64_t v = rank_value(fb[i], fi[i]);
-    const uint32_t slot = atomicAdd(&start[hdigit_v(v)], 1u);
-    tv[slot] = v;
-    tb[slot] = fb[i];
-  }
-  group_sync(NT);
-  // start[d] now ends bin d's range of tv; rank each entry inside it
-  for (int i = tid; i < n; i += NT) {
-    const uint64_t v = tv[i];
-    const uint32_t d = hdigit_v(v);
+  // start[d] now ends bin d's range of tv
+  for (int i = tid; i < above; i += NT) {
+    const uint64_t x = tv[i];
+    const uint32_t d = hdigit_v(x);
     const int hi = (int)start[d];
-    const int lo = hi - (int)cnt[d];
-    int pos = lo;
-    for (int j = lo; j < hi; ++j) pos += tv[j] > v;
-    idx_out[pos] = (int32_t)~(uint32_t)v;
+    int pos = hi - (int)hist[d];
+    for (int j = pos; j < hi; ++j) pos += tv[j] > x;
+    idx_out[pos] = (int32_t)~(uint32_t)x;
     if (val_out) val_out[pos] = __uint_as_float(tb[i]);
   }
-  for (int k = n + tid; k < K; k += NT) {
+  rank_boundary<NT>(bl_v, bl_b, cnt, K - above, [&](int rank, uint64_t x, uint32_t xb) {
+    idx_out[above + rank] = (int32_t)~(uint32_t)x;
+    if (val_out) val_out[above + rank] = __uint_as_float(xb);
+  });
+  for (int k = min(total, K) + tid; k < K; k += NT) {
     idx_out[k] = -1;
     if (val_out) val_out[k] = __uint_as_float(kNegInfBits);
   }
   group_sync(NT);
 }
 
-// Order the winners and write the row: few winners go to the counting sort of
-// sort_and_write (two barriers), more to hist_write_sorted.
-template <int NT>
-__device__ __forceinline__ void hist_write_row(const uint32_t* fb, const uint32_t* fi, int n,
-                                               int K, uint32_t* cnt, uint32_t* start,
-                                               SelectScratch& sc, uint64_t* tv, uint32_t* tb,
-                                               int32_t* idx_out, float* val_out) {
-  if (n <= 2 * NT) sort_and_write<NT>(fb, fi, n, K, tv, tb, idx_out, val_out);
-  else hist_write_sorted<NT>(fb, fi, n, K, cnt, start, sc, tv, tb, idx_out, val_out);
+// Exact top K of register-held entries as one unordered candidate list of
+// exactly K entries (cbits / cidx; unused entries -inf / -1), after
+// hist_scan on their exact histogram.  When entries were dropped, the K-th
+// largest rank value raises *row_thr (atomic max): every entry of the row's
+// top K is at least that.
+template <int NT, int E>
+__device__ void place_publish(const uint64_t (&v)[E], const uint32_t (&bits)[E], int nk,
+                              uint32_t* start, int K, SelectScratch& sc, uint64_t* bl_v,
+                              uint32_t* bl_b, uint32_t* cbits, int32_t* cidx,
+                              unsigned long long* row_thr) {
+  const uint32_t b = sc.bcast[0];
+  const int above = (int)sc.bcast[1];
+  const int cnt = (int)sc.bcast[2];
+  const int total = (int)sc.bcast[3];
+  classify(v, bits, nk, b, (uint32_t)above, start, bl_v, bl_b,
+           [&](uint64_t x, uint32_t xb, uint32_t, uint32_t slot) {
+             cbits[slot] = xb;
+             cidx[slot] = (int32_t)~(uint32_t)x;
+           });
+  if (threadIdx.x == 0) bl_v[cnt] = 0ull;
+  group_sync(NT);
+  const int r = K - above;
+  rank_boundary<NT>(bl_v, bl_b, cnt, r, [&](int rank, uint64_t x, uint32_t xb) {
+    cbits[above + rank] = xb;
+    cidx[above + rank] = (int32_t)~(uint32_t)x;
+    if (rank == r - 1) atomicMax(row_thr, (unsigned long long)x);
+  });
+  for (int k = min(total, K) + (int)threadIdx.x; k < K; k += NT) {
+    cbits[k] = kNegInfBits;
+    cidx[k] = -1;
+  }
+}
+
+// Load a filter buffer's n entries into registers (entry i = tid + k * NT).
+template <int NT, int E>
+__device__ __forceinline__ int load_buffer(const uint32_t* fb, const uint32_t* fi, int n,
+                                           uint64_t (&v)[E], uint32_t (&bits)[E]) {
+  const int nk = (n + NT - 1) / NT;
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int i = (int)threadIdx.x + k * NT;
+    v[k] = 0ull;
+    bits[k] = 0u;
+    if (k < nk && i < n) {
+      bits[k] = fb[i];
+      v[k] = rank_value(bits[k], fi[i]);
+    }
+  }
+  return nk;
 }
 
 // Merge published candidate lists (list i at bits/index + slot_of(i) *
-// stride, K entries each, unused entries -inf) into one ordered output row.
-// Every thread keeps U loads in flight; entries below the row threshold are
-// dropped on arrival, the rest go into a histogram-tracked filter (radix
-// compaction and a recount only if the buffer of cap entries would
-// overflow); then the exact winners are taken from the histogram and written
-// in order.  hist/chist: the filter histograms (clobbered); start: kHBins
-// words; tv/tb: max(64, next_pow2(K)) + 1 entries.  Resets *row_thr to zero
-// for the next call.
-template <int NT, class SlotOf>
-__device__ void hist_merge(int nslots, SlotOf slot_of, const uint32_t* cand_bits,
-                           const int32_t* cand_idx, int64_t stride, int K,
-                           unsigned long long* row_thr, FilterState& fs, uint32_t* fb, uint32_t* fi,
-                           int cap, uint32_t* hist, uint32_t* chist, uint32_t* start,
-                           SelectScratch& sc, uint64_t* tv, uint32_t* tb, int32_t* idx_out,
-                           float* val_out) {
-  constexpr int U = 8;
+// stride, K entries each, unused entries -inf) into one ordered output row,
+// when all nslots * K entries fit in registers (E per thread).  Every thread
+// issues all its loads at once (the row threshold is read meanwhile);
+// entries below the threshold are dropped, the rest counted in hist, and the
+// exact winners are placed in order.  Resets *row_thr to zero for the next
+// call.  Returns false, having done nothing but the reset, when the boundary
+// bin is too crowded (heavy ties): the caller then merges another way.
+template <int NT, int E, class SlotOf>
+__device__ bool hist_merge_regs(int nslots, SlotOf slot_of, const uint32_t* cand_bits,
+                                const int32_t* cand_idx, int64_t stride, int K,
+                                unsigned long long* row_thr, uint32_t* hist, uint32_t* start,
+                                SelectScratch& sc, uint64_t* tv, uint32_t* tb, uint64_t* bl_v,
+                                uint32_t* bl_b, int32_t* idx_out, float* val_out) {
   const int tid = threadIdx.x;
-  hist_clear<NT>(hist, chist);
+  const int total = nslots * K;
+  uint64_t v[E];
+  uint32_t bits[E];
+  uint32_t index[E];
+  int i0 = tid / K, e0 = tid - i0 * K;  // list and entry of f = tid, advanced by NT
+  const int di = NT / K, de = NT - di * K;
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    bits[k] = kNegInfBits;
+    index[k] = 0u;
+    if (k * NT + tid < total) {
+      const int64_t off = slot_of(i0) * stride + e0;
+      bits[k] = __ldcg(cand_bits + off);
+      index[k] = (uint32_t)__ldcg(cand_idx + off);
+    }
+    i0 += di;
+    e0 += de;
+    if (e0 >= K) {
+      e0 -= K;
+      ++i0;
+    }
+  }
+  for (int i = tid; i < kHBins; i += NT) hist[i] = 0u;
   if (tid == 0) {
     const unsigned long long t = __ldcg(row_thr);
-    fs.thr = t ? t - 1 : 0ull;  // keep v >= t
-    fs.count = 0;
+    *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = t ? t - 1 : 0ull;  // keep v >= t
     *row_thr = 0ull;
   }
   group_sync(NT);
-  const int total = nslots * K;
-  for (int f0 = 0; f0 < total; f0 += NT * U) {
-    uint32_t bits[U], index[U];
+  const unsigned long long thr = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
+  int nk = 0;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int f = f0 + u * NT + tid;
-      bits[u] = kNegInfBits;
-      index[u] = 0xFFFFFFFFu;
-      if (f < total) {
-        const int i = f / K;
-        const int e = f - i * K;
-        const int64_t off = slot_of(i) * stride + e;
-        bits[u] = __ldcg(cand_bits + off);
-        index[u] = (uint32_t)__ldcg(cand_idx + off);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-      filter_offer_h(fs, fb, fi, hist, chist, bits[u], index[u], index[u] != 0xFFFFFFFFu);
-    group_sync(NT);
-    if (f0 + NT * U < total && fs.count > cap - NT * U) {
-      filter_compact<NT>(fs, fb, fi, K, sc);
-      hist_rebuild<NT>(fs, fb, fi, hist, chist);
-    }
+  for (int k = 0; k < E; ++k) {
+    const uint64_t x = rank_value(bits[k], index[k]);
+    v[k] = x > thr ? x : 0ull;
+    if (v[k]) atomicAdd(&hist[hdigit_v(v[k])], 1u);
+    if (k * NT < total) nk = k + 1;
   }
-  const int kk = hist_winners<NT>(fs, fb, fi, hist, K, sc, tv, tb);
-  hist_write_row<NT>(fb, fi, kk, K, hist, start, sc, tv, tb, idx_out, val_out);
+  group_sync(NT);
+  hist_scan<NT>(hist, start, (uint32_t)K, sc);
+  if (sc.bcast[0] != 0xFFFFFFFFu && sc.bcast[2] > (uint32_t)kBoundaryMax) return false;
+  place_ordered<NT, E>(v, bits, nk, hist, start, K, sc, tv, tb, bl_v, bl_b, idx_out, val_out);
+  return true;
 }
 
 }  // namespace idx

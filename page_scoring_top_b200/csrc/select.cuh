@@ -435,25 +435,27 @@ __device__ void merge_candidates(int nslots, SlotOf slot_of, const uint32_t* can
   IDX_TRACE(5);
 }
 
-// All threads of the group: publish this CTA's stores, then count one arrival
-// on *counter.  Returns true (to every thread) in the CTA that arrives last
-// (the expected-th arrival); that CTA also resets the counter to zero.
+// All threads of the group: count one arrival on *counter once this CTA's
+// global stores are visible GPU-wide.  Returns true (to every thread) in the
+// CTA that arrives last (the expected-th arrival), which also resets the
+// counter to zero; its reads of the other CTAs' stores are ordered after
+// theirs.  The barrier orders every thread's stores before thread 0's
+// release fence and arrival; thread 0's acquire fence and the second barrier
+// order the other CTAs' stores before this CTA's later reads.
 template <int NT>
 __device__ bool arrive_last(int32_t* counter, int expected, int* s_flag) {
-  __threadfence();
   group_sync(NT);
   if (threadIdx.x == 0) {
-    const int old = atomicAdd(counter, 1);
-    *s_flag = (old == expected - 1);
-  }
-  group_sync(NT);
-  const bool last = *s_flag != 0;
-  if (last) {
     __threadfence();
-    if (threadIdx.x == 0) *counter = 0;
+    const bool last = atomicAdd(counter, 1) == expected - 1;
+    if (last) {
+      *counter = 0;
+      __threadfence();
+    }
+    *s_flag = last;
   }
   group_sync(NT);
-  return last;
+  return *s_flag != 0;
 }
 
 }  // namespace idx
