@@ -35,11 +35,15 @@ METRIC = "pages scored+selected/sec and HBM GB/s vs 8 TB/s at B=32,N=65536,K=256
 UNIT = "pages/s"
 WORKLOAD = "ragged_decode"
 NOMINAL_HBM_GBS = 8000.0
+# The one kernel a step launches: tcgen05 scoring (D=128, query rows unrolled
+# to 16), fused with the histogram-driven top-K select.
+KERNEL = "decode_tc_kernel<D=128,NC=16,fused,hist>"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per valid page of the fused decode kernel, from the ncu capture
-# summarised in profiles/ (dram__bytes_read.sum + dram__bytes_write.sum per
-# launch / pages per launch); None until a capture of the current kernel exists.
-NCU_TRAFFIC_BYTES_PER_PAGE = None  # the kernel changed after the last capture
+# summarised in profiles/decode_fused_ragged_decode.md: (301.28 MB read +
+# 3.95 MB written) per launch / 1,175,731 pages.  Set to None whenever the
+# kernel changes until it is captured again.
+NCU_TRAFFIC_BYTES_PER_PAGE = 259.6
 
 
 def parse():
@@ -281,8 +285,8 @@ def run_ours(args):
     if rc != 0:
         raise RuntimeError("device status %d after the timed region" % bits)
 
-    # Roofline of the dominant (only) kernel: the fused decode kernel, one
-    # launch per step on `stream`, timed by the events above.
+    # Roofline of the dominant (only) kernel: the fused tensor-core decode
+    # kernel, one launch per step on `stream`, timed by the events above.
     launch_s = (ms / args.steps) * 1e-3
     achieved = nbytes / launch_s / 1e9
     peak, peak_src = measured_peak()
@@ -312,7 +316,7 @@ def run_ours(args):
             "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "kernel": "decode_kernel<128,1,fused>"},
+                         "kernel": KERNEL},
             "gpu_launches": args.steps,
             "clocks": clocks,
             "e2e": e2e,

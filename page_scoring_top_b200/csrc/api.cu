@@ -61,7 +61,8 @@ int check_score_args(const idx_ctx* ctx, const uint16_t* q, const uint16_t* c, i
   if (ldc_b < (int64_t)N * D || (ldc_b % 8) != 0) return IDX_EINVAL;
   if ((D % 8) != 0 || D > 256) return IDX_EUNSUPPORTED;
   if ((int64_t)B * T > ctx->max_rows || N > ctx->max_n) return IDX_ENOWORKSPACE;
-  if ((int64_t)B * N > INT32_MAX) return IDX_EUNSUPPORTED;
+  // page counts, plus the per-request work charge of the fused split, are ints
+  if ((int64_t)B * ((int64_t)N + 1024) > INT32_MAX) return IDX_EUNSUPPORTED;
   return IDX_OK;
 }
 

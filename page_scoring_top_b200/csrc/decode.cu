@@ -154,11 +154,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   }
   length_prefix(a, s_off, s_wsum, kDecodeThreads);
   __syncthreads();
-  const int P = s_off[B];
-  int Lc = (P + G - 1) / G;
-  if (FUSED) Lc = Lc < kLMin ? kLMin : Lc;
-  Lc = Lc < 1 ? 1 : Lc;
-  const int nchunks = (P + Lc - 1) / Lc;
+  const Chunking ch = make_chunking(s_off, B, G, FUSED ? kSegmentPages : 0, FUSED ? kLMin : 1);
+  const int nchunks = ch.nchunks;
 
   // ------------------------------------------------------------------ producer
   // Lanes 0..kProducerLanes-1 issue the stages round-robin (stage k by lane
@@ -170,12 +167,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
       const uint64_t pol = policy_evict_first();
       uint32_t stage = 0;
       for (int j = g; j < nchunks; j += G) {
-        const int cb = j * Lc, ce = min(cb + Lc, P);
-        const int b_last = row_of(s_off, B, ce - 1);
-        for (int b = row_of(s_off, B, cb); b <= b_last; ++b) {
-          if (s_off[b + 1] == s_off[b]) continue;
-          const int p0 = snap_local(s_off, b, cb);
-          const int np = snap_local(s_off, b, ce) - p0;
+        const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
+        const int b_last = ch.row(ce - 1);
+        for (int b = ch.row(cb); b <= b_last; ++b) {
+          if (ch.len(b) == 0) continue;
+          const int p0 = ch.snap(b, cb);
+          const int np = ch.snap(b, ce) - p0;
           const uint16_t* src = a.c + (int64_t)b * a.ldc_b + (int64_t)p0 * D;
           for (int sp = 0; sp < np; sp += kStagePages, ++stage) {
             if ((int)(stage % kProducerLanes) != lane) continue;
@@ -232,12 +229,12 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   uint32_t stage = 0;
 
   for (int j = g; j < nchunks; j += G) {
-    const int cb = j * Lc, ce = min(cb + Lc, P);
-    const int b_last = row_of(s_off, B, ce - 1);
-    for (int b = row_of(s_off, B, cb); b <= b_last; ++b) {
-      if (s_off[b + 1] == s_off[b]) continue;
-      const int p0 = snap_local(s_off, b, cb);
-      const int np = snap_local(s_off, b, ce) - p0;  // may be 0
+    const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
+    const int b_last = ch.row(ce - 1);
+    for (int b = ch.row(cb); b <= b_last; ++b) {
+      if (ch.len(b) == 0) continue;
+      const int p0 = ch.snap(b, cb);
+      const int np = ch.snap(b, ce) - p0;  // may be 0
       if (FUSED) {
         fused_begin<HIST>(fsel, T);
         group_sync(kConsumers);
@@ -332,7 +329,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
         }
       }
       if (FUSED)
-        fused_finalize<HIST>(fsel, a, T, b, j, s_off[b] / Lc, (s_off[b + 1] - 1) / Lc);
+        fused_finalize<HIST>(fsel, a, T, b, j, ch.first(b), ch.last(b));
     }
   }
 }
@@ -348,8 +345,9 @@ int decode_fused_max_k(int T) {
 }
 
 int64_t decode_fused_slots(int64_t B, int64_t T, int64_t N, int grid) {
-  // The fused chunk length is max(ceil(P/grid), kLMin), so there are at most
-  // `grid` chunks; the pair (chunk j, request b) owns slot (j + b) per token.
+  // The fused chunk length is at least ceil(virtual pages / grid), so there
+  // are at most `grid` chunks; the pair (chunk j, request b) owns slot (j + b)
+  // per token.
   (void)N;
   return ((int64_t)grid + 1 + B) * T;
 }

@@ -180,11 +180,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int P = s_off[B];
-  int Lc = (P + G - 1) / G;
-  if (FUSED) Lc = Lc < kTcLMin ? kTcLMin : Lc;
-  Lc = Lc < 1 ? 1 : Lc;
-  const int nchunks = (P + Lc - 1) / Lc;
+  const Chunking ch = make_chunking(s_off, B, G, FUSED ? kSegmentPages : 0, FUSED ? kTcLMin : 1);
+  const int nchunks = ch.nchunks;
 
   if (warp == kTcProducerWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -194,12 +191,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t tile = 0;
       int64_t last = -1;  // last tile this lane issued
       for (int j = g; j < nchunks; j += G) {
-        const int cb = j * Lc, ce = min(cb + Lc, P);
-        const int b_last = row_of(s_off, B, ce - 1);
-        for (int b = row_of(s_off, B, cb); b <= b_last; ++b) {
-          if (s_off[b + 1] == s_off[b]) continue;
-          const int p0 = snap_local(s_off, b, cb);
-          const int nps = snap_local(s_off, b, ce) - p0;
+        const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
+        const int b_last = ch.row(ce - 1);
+        for (int b = ch.row(cb); b <= b_last; ++b) {
+          if (ch.len(b) == 0) continue;
+          const int p0 = ch.snap(b, cb);
+          const int nps = ch.snap(b, ce) - p0;
           for (int r0 = 0; r0 < nps; r0 += kTcTile, ++tile) {
             if ((int)(tile % (uint32_t)lanes) != lane) continue;
             const int slot = (int)(tile % (uint32_t)nst);
@@ -241,12 +238,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t tile = 0;
     int seg = 0;
     for (int j = g; j < nchunks; j += G) {
-      const int cb = j * Lc, ce = min(cb + Lc, P);
-      const int b_last = row_of(s_off, B, ce - 1);
-      for (int b = row_of(s_off, B, cb); b <= b_last; ++b) {
-        if (s_off[b + 1] == s_off[b]) continue;
-        const int p0 = snap_local(s_off, b, cb);
-        const int nps = snap_local(s_off, b, ce) - p0;
+      const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
+      const int b_last = ch.row(ce - 1);
+      for (int b = ch.row(cb); b <= b_last; ++b) {
+        if (ch.len(b) == 0) continue;
+        const int p0 = ch.snap(b, cb);
+        const int nps = ch.snap(b, ce) - p0;
         if (nps <= 0) continue;
         // The previous request's MMAs must be done reading the query rows.
         if (seg > 0 && lane == 0) mbar_wait_bounded(q_free, (uint32_t)(seg - 1) & 1, s_abort, a.status);
@@ -298,21 +295,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (!FUSED) score_padding(a, s_off, g, G);
     else fused_empty_rows(a, s_off, g, G);
     const int rows = T * Q;
-    const int check_tiles = FUSED ? 2 * fused_rounds(L.cap, a.K) : 1;
-    const int compact_at = FUSED ? fused_compact_at<HIST>(L.cap, a.K) : 0;
+    // Filter checks: a tile appends at most 128 entries per token, so after a
+    // check that leaves `room` free entries the next one comes within
+    // room / 128 tiles.  With the histogram the compaction is only the
+    // overflow guard; without it, it also raises the threshold.
+    const int compact_at = FUSED ? (HIST ? L.cap - 2 * kTcTile : fused_compact_at<HIST>(L.cap, a.K)) : 0;
     uint32_t tile = 0;
     for (int j = g; j < nchunks; j += G) {
-      const int cb = j * Lc, ce = min(cb + Lc, P);
-      const int b_last = row_of(s_off, B, ce - 1);
-      for (int b = row_of(s_off, B, cb); b <= b_last; ++b) {
-        if (s_off[b + 1] == s_off[b]) continue;
-        const int p0 = snap_local(s_off, b, cb);
-        const int nps = snap_local(s_off, b, ce) - p0;
+      const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
+      const int b_last = ch.row(ce - 1);
+      for (int b = ch.row(cb); b <= b_last; ++b) {
+        if (ch.len(b) == 0) continue;
+        const int p0 = ch.snap(b, cb);
+        const int nps = ch.snap(b, ce) - p0;
         if (FUSED) {
           fused_begin<HIST>(fsel, T);
           group_sync(kTcEpi);
         }
         const int ntl = (nps + kTcTile - 1) / kTcTile;
+        int next_check = FUSED ? (L.cap - a.K) / kTcTile - 1 : 0;
         for (int tt = 0; tt < ntl; ++tt, ++tile) {
           if ((int)(tile & 1) == wg) {
             const int acc = (int)(tile % kTcAcc);
@@ -331,33 +332,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int row = tt * kTcTile + quad * 32 + lane;
             const bool mine = row < nps;
             const int page = p0 + row;
-            // head-sums in head order, one token after another
-            float s = 0.f;
-            int h = 0, t = 0;
+            // head-sums in head order, one token after another (starting from
+            // -0, which adds exactly: the same bits in both modes)
+            if (FUSED) {
+              constexpr int TM = HIST ? 1 : kMaxFusedT;
+              float st[TM];
 #pragma unroll
-            for (int col = 0; col < NC; ++col) {
-              if (col < rows) {
-                s = h == 0 ? __uint_as_float(v[col]) : s + __uint_as_float(v[col]);
-                if (++h == Q) {
-                  if (FUSED) {
-                    fused_offer<HIST>(fsel, t, __float_as_uint(s), (uint32_t)page, mine);
-                  } else if (mine) {
-                    a.scores[((int64_t)b * T + t) * N + page] = s;
+              for (int t = 0; t < TM; ++t) st[t] = -0.f;
+#pragma unroll
+              for (int col = 0; col < NC; ++col) {
+                if (col < rows) {
+                  const float x = __uint_as_float(v[col]);
+#pragma unroll
+                  for (int t = 0; t < TM; ++t)
+                    if (col >= t * Q && col < t * Q + Q) st[t] += x;
+                }
+              }
+#pragma unroll
+              for (int t = 0; t < TM; ++t)
+                if (t < T) fused_offer<HIST>(fsel, t, __float_as_uint(st[t]), (uint32_t)page, mine);
+            } else {
+              float s = -0.f;
+              int h = 0, t = 0;
+#pragma unroll
+              for (int col = 0; col < NC; ++col) {
+                if (col < rows) {
+                  s += __uint_as_float(v[col]);
+                  if (++h == Q) {
+                    if (mine) a.scores[((int64_t)b * T + t) * N + page] = s;
+                    s = -0.f;
+                    h = 0;
+                    ++t;
                   }
-                  h = 0;
-                  ++t;
                 }
               }
             }
-            // every other tile, one warp lifts the threshold from the histogram
-            if (HIST && (int)((tile >> 1) & 7) == quad) fused_raise(fsel, a.K);
+            // twice per 8 tiles (once per warpgroup), one warp lifts the
+            // threshold from the histogram
+            if (HIST && (tile & 7) == (wg ? 5u : 0u) && (int)((tile >> 3) & 3) == quad)
+              fused_raise(fsel, a.K);
           }
-          if (FUSED && ((tt + 1) % check_tiles == 0 || tt + 1 == ntl)) {
+          if (FUSED && (tt == next_check || tt + 1 == ntl)) {
             group_sync(kTcEpi);  // every offer so far is complete
-            fused_check<HIST>(fsel, T, a.K, compact_at);
+            next_check = tt + max(1, fused_check<HIST>(fsel, T, a.K, compact_at) / kTcTile);
           }
         }
-        if (FUSED) fused_finalize<HIST>(fsel, a, T, b, j, s_off[b] / Lc, (s_off[b + 1] - 1) / Lc);
+        if (FUSED) fused_finalize<HIST>(fsel, a, T, b, j, ch.first(b), ch.last(b));
       }
     }
   }

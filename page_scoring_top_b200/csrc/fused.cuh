@@ -19,6 +19,10 @@ namespace idx {
 
 constexpr int kSelThreads = 256;  // threads 0..255 run every select step
 constexpr int kMaxFusedT = 4;
+// Virtual pages charged per request in fused mode: about what a segment-end
+// select step costs in streaming time (a few microseconds at one SM's share
+// of HBM bandwidth, minus what the stage ring absorbs).
+constexpr int kSegmentPages = 512;
 
 // Shared-memory state of the fused select (pointers into the kernel's layout).
 struct FusedSel {
@@ -65,15 +69,28 @@ __device__ __forceinline__ void fused_raise(const FusedSel& f, int K) {
 }
 
 // Overflow guard at a check point (all select threads, after a barrier that
-// completed every offer): compact a filter holding more than compact_at.
+// completed every offer): compact each filter holding more than compact_at.
+// Every thread reads the counts before a second barrier, so all of them take
+// the same decision even when fast warps go back to offering right after.
+// Returns the smallest free room (cap - count) over the filters afterwards.
 template <bool HIST>
-__device__ __forceinline__ void fused_check(const FusedSel& f, int T, int K, int compact_at) {
+__device__ __forceinline__ int fused_check(const FusedSel& f, int T, int K, int compact_at) {
+  uint32_t over = 0;
+  int used = 0;
+  for (int t = 0; t < T; ++t) {
+    const int n = f.fst[t].count;
+    if (n > compact_at) over |= 1u << t;
+    else used = max(used, n);
+  }
+  group_sync(kSelThreads);
   for (int t = 0; t < T; ++t)
-    if (f.fst[t].count > compact_at) {
+    if (over >> t & 1u) {
       uint32_t* fb = f.fbuf + t * 2 * f.cap;
       filter_compact<kSelThreads>(f.fst[t], fb, fb + f.cap, K, *f.sc);
       if (HIST) hist_rebuild<kSelThreads>(f.fst[0], f.fbuf, f.fbuf + f.cap, f.hist, f.hist + kHBins);
+      used = max(used, min(K, f.fst[t].count));
     }
+  return f.cap - used;
 }
 
 // Check period (in rounds of 256 offers per token) and compaction mark: a
@@ -242,27 +259,58 @@ __device__ __forceinline__ void length_prefix(const DecodeArgs& a, int* s_off, u
   }
 }
 
-// First request b whose pages extend past global page gp (s_off[b+1] > gp).
-__device__ __forceinline__ int row_of(const int* s_off, int B, int gp) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (s_off[mid + 1] > gp) hi = mid;
-    else lo = mid + 1;
-  }
-  return lo;
-}
+// Work split of a decode launch.  The valid pages of the batch are laid end
+// to end; in fused mode every request is also charged W pages of virtual
+// work up front (a segment end costs a select step, which a CTA whose chunk
+// ends a request pays while its stream waits), and the resulting virtual
+// page range is cut into equal chunks, one per CTA.  Request b occupies the
+// virtual range [voff(b), voff(b+1)), its real pages the last len(b) of it.
+// Each (chunk, request) piece is a segment; its real pages run from
+// snap(b, chunk start) to snap(b, chunk end), both multiples of 32, so the
+// arithmetic of a page's score does not depend on how the batch was cut.
+struct Chunking {
+  const int* s_off;  // prefix sums of the clamped lengths
+  int B, W, PV, Lc, nchunks;
 
-// Local page index in request b of the chunk boundary at global page x, snapped
-// down to a multiple of 32 pages (or clamped to the row's ends).  Every
-// segment then starts at a request-local page index that is a multiple of 32,
-// so the arithmetic of a page's score depends on the page alone, not on how
-// the batch was cut into chunks.
-__device__ __forceinline__ int snap_local(const int* s_off, int b, int x) {
-  const int len = s_off[b + 1] - s_off[b];
-  const int r = x - s_off[b];
-  if (r >= len) return len;
-  return r <= 0 ? 0 : (r & ~31);
+  __device__ __forceinline__ int voff(int b) const { return s_off[b] + b * W; }
+  __device__ __forceinline__ int len(int b) const { return s_off[b + 1] - s_off[b]; }
+  // First request whose virtual range extends past x.
+  __device__ __forceinline__ int row(int x) const {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (voff(mid + 1) > x) hi = mid;
+      else lo = mid + 1;
+    }
+    return lo;
+  }
+  // Real page of request b at virtual position x, snapped down to 32 (or
+  // clamped to the row's ends).
+  __device__ __forceinline__ int snap(int b, int x) const {
+    const int n = len(b);
+    const int r = x - voff(b) - W;
+    if (r >= n) return n;
+    return r <= 0 ? 0 : (r & ~31);
+  }
+  // Chunks holding a segment of request b: first0(b) .. last(b).
+  __device__ __forceinline__ int first(int b) const { return voff(b) / Lc; }
+  __device__ __forceinline__ int last(int b) const { return (voff(b + 1) - 1) / Lc; }
+  __device__ __forceinline__ int chunk_begin(int j) const { return j * Lc; }
+  __device__ __forceinline__ int chunk_end(int j) const { return min(j * Lc + Lc, PV); }
+};
+
+// s_off must be complete (after the barrier that ends length_prefix).
+__device__ __forceinline__ Chunking make_chunking(const int* s_off, int B, int G, int W, int lmin) {
+  Chunking c;
+  c.s_off = s_off;
+  c.B = B;
+  c.W = W;
+  c.PV = s_off[B] + B * W;
+  int Lc = (c.PV + G - 1) / G;
+  Lc = Lc < lmin ? lmin : Lc;
+  c.Lc = Lc < 1 ? 1 : Lc;
+  c.nchunks = (c.PV + c.Lc - 1) / c.Lc;
+  return c;
 }
 
 }  // namespace idx
