@@ -157,6 +157,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t tcols = 32;
   while (tcols < (uint32_t)(kTcAcc * np)) tcols <<= 1;
 
+  // The next launch may start taking SMs as this grid's CTAs finish; the
+  // shared-memory and TMEM setup below overlaps the previous grid's tail,
+  // and nothing in global memory is touched before griddep_wait.
+  griddep_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&full[s], 1);
@@ -175,6 +179,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   for (int i = tid; i < np * D * 2 / 16; i += kTcThreads)
     reinterpret_cast<uint4*>(qop)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
+  griddep_wait();
   length_prefix(a, s_off, s_wsum, kTcThreads);
   tc_fence_before();
   __syncthreads();
@@ -395,8 +400,19 @@ cudaError_t launch_tc(const CUtensorMap& mt, const CUtensorMap& ms, const Decode
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NC, FUSED, HIST>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<D, NC, FUSED, HIST><<<grid, kTcThreads, smem, stream>>>(mt, ms, a);
-  return cudaGetLastError();
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream: its setup overlaps that kernel's tail, its global reads wait.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<D, NC, FUSED, HIST>, mt, ms, a);
 }
 
 template <int D, bool FUSED, bool HIST>
