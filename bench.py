@@ -10,6 +10,12 @@ request are written.  The metric is valid pages scored+selected per second
 (whole job) and the HBM bandwidth that implies.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload ragged_decode|prefill_chunk|batch_decode_bias|tiny_decode]
+
+The default workload is the headline one above.  The others are the indexer's
+remaining workloads, for profiling: a prefill chunk (B=4, T=16, Q=8, N=131072,
+K=512; every token row of 131072 pages selects its top 512) counts one unit per
+(token row, page).
 For N > 1 launch under torch.distributed.run: requests are sharded across ranks
 (each rank owns its batch; no collective on the data path), timing is the max
 over ranks.  ``--impl reference`` times the CPU oracle (single-threaded C) on
@@ -38,6 +44,7 @@ NOMINAL_HBM_GBS = 8000.0
 # The one kernel a step launches: tcgen05 scoring (D=128, query rows unrolled
 # to 16), fused with the histogram-driven top-K select.
 KERNEL = "decode_tc_kernel<D=128,NC=16,fused,hist>"
+PREFILL_KERNEL = "prefill_kernel<Q=8> (tcgen05 score of a 16-token chunk)"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per valid page of the fused decode kernel, from the ncu capture
 # summarised in profiles/decode_fused_ragged_decode.md: (301.28 MB read +
@@ -56,6 +63,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=("ragged_decode", "prefill_chunk", "batch_decode_bias", "tiny_decode"))
     return ap.parse_args()
 
 
@@ -66,12 +75,12 @@ def dist_env():
     return rank, world, local
 
 
-def workload_inputs(rank):
+def workload_inputs(rank, name=WORKLOAD):
     from page_scoring_top_b200 import dist as pdist
     from page_scoring_top_b200 import synth
-    spec = dict(synth.WORKLOADS[WORKLOAD])
+    spec = dict(synth.WORKLOADS[name])
     seed = pdist.rank_seed(spec["seed"], rank)
-    return synth.workload(WORKLOAD, seed=seed), spec, seed
+    return synth.workload(name, seed=seed), spec, seed
 
 
 def algorithmic_bytes(lengths, B, T, Q, D, K, with_values):
@@ -234,11 +243,12 @@ def run_ours(args):
         pg = dist
     from page_scoring_top_b200 import binding
 
-    d, spec, seed = workload_inputs(rank)
+    d, spec, seed = workload_inputs(rank, args.workload)
     B, T, Q, D = d["q"].shape
     N = d["c"].shape[1]
     K = spec["K"]
     pages, nbytes = algorithmic_bytes(d["lengths"], B, T, Q, D, K, with_values=False)
+    units = pages * T  # (token row, valid page) pairs scored and selected
 
     q = torch.from_numpy(d["q"].view(np.int16)).to(dev)
     c = torch.from_numpy(d["c"].view(np.int16)).to(dev)
@@ -278,26 +288,50 @@ def run_ours(args):
     barrier()
     ms = ev0.elapsed_time(ev1)
     from page_scoring_top_b200 import dist as pdist
-    ms_max, total_pages = pdist.reduce_timing(ms, pages, device=dev)
+    ms_max, total_pages = pdist.reduce_timing(ms, units, device=dev)
     ms_per_step = ms_max / args.steps
     value = total_pages * args.steps / (ms_max * 1e-3)
     rc, bits = binding.idx_get_status(ctx)
     if rc != 0:
         raise RuntimeError("device status %d after the timed region" % bits)
 
-    # Roofline of the dominant (only) kernel: the fused tensor-core decode
-    # kernel, one launch per step on `stream`, timed by the events above.
-    launch_s = (ms / args.steps) * 1e-3
-    achieved = nbytes / launch_s / 1e9
+    # Roofline of the dominant kernel.  Decode: the fused tensor-core decode
+    # kernel is the step's only launch, timed by the events above.  Prefill:
+    # the step is the tcgen05 score kernel then the top-K kernel; the score
+    # kernel (centroid_score alone) is timed the same way on the same stream.
     peak, peak_src = measured_peak()
-    traffic = None if NCU_TRAFFIC_BYTES_PER_PAGE is None else NCU_TRAFFIC_BYTES_PER_PAGE * pages
+    kernel, traffic = KERNEL, None
+    if args.workload == WORKLOAD and NCU_TRAFFIC_BYTES_PER_PAGE is not None:
+        traffic = NCU_TRAFFIC_BYTES_PER_PAGE * pages
+    launch_s = (ms / args.steps) * 1e-3
+    score_bytes = nbytes
+    tensor = None
+    if T > 1:
+        kernel = PREFILL_KERNEL
+        scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
+        for _ in range(args.warmup):
+            binding.centroid_score(ctx, q, c, ln, scores, stream=stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            binding.centroid_score(ctx, q, c, ln, scores, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        launch_s = e0.elapsed_time(e1) / args.steps * 1e-3
+        # algorithmic bytes of the score kernel: valid centroids + q read,
+        # every score written (padding included)
+        score_bytes = pages * D * 2 + B * T * Q * D * 2 + B * T * N * 4
+        flops = 2.0 * pages * T * Q * D
+        tensor = {"achieved_tflops": flops / launch_s / 1e12, "score_kernel_us": launch_s * 1e6}
+    achieved = score_bytes / launch_s / 1e9
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.workload == WORKLOAD:
         e2e = measure_e2e(binding, ctx, d, K, dev, stream, args.e2e_steps, barrier, pg)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         rate, sample = cpu_oracle_rate(d, K, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
 
@@ -307,8 +341,9 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": B, "T": T, "Q": Q, "D": D, "N": N, "K": K,
-                       "len_dist": "uniform 1024..65536", "seed": seed,
+            "config": {"workload": args.workload, "B": B, "T": T, "Q": Q, "D": D, "N": N, "K": K,
+                       "len_dist": ("uniform 1024..65536" if args.workload == WORKLOAD
+                                    else "all pages valid"), "seed": seed,
                        "pages_per_step_per_gpu": pages, "bytes_per_step_per_gpu": nbytes,
                        "parallelism": "dp%d (requests sharded, no data-path collective)" % world,
                        "l2": "inputs larger than L2 (%.1f MB of centroids per step vs 126 MB); "
@@ -316,9 +351,10 @@ def run_ours(args):
             "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "kernel": KERNEL},
-            "gpu_launches": args.steps,
+                         "kernel": kernel},
+            "gpu_launches": args.steps * (2 if T > 1 else 1),
             "clocks": clocks,
+            "tensor": tensor,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

@@ -426,7 +426,10 @@ __device__ void merge_candidates(int nslots, SlotOf slot_of, const uint32_t* can
 #pragma unroll
     for (int u = 0; u < U; ++u) filter_offer(fs, fb, fi, bits[u], index[u], index[u] != 0xFFFFFFFFu);
     group_sync(NT);
-    if (fs.count > cap - NT * U) filter_compact<NT>(fs, fb, fi, K, sc);
+    // every thread reads the count before anyone offers again: one decision
+    const int n = fs.count;
+    group_sync(NT);
+    if (n > cap - NT * U) filter_compact<NT>(fs, fb, fi, K, sc);
   }
   IDX_TRACE(3);
   if (fs.count > 2 * NT) filter_compact<NT>(fs, fb, fi, K, sc);

@@ -133,7 +133,10 @@ __global__ void __launch_bounds__(NT) topk_chunk_kernel(const TopkArgs a) {
       for (int k = 0; k < 4; ++k)
         filter_offer(fs, fb, fi, w[k], (uint32_t)(c0 + e0 + k), e0 + k < n);
       group_sync(NT);
-      if (fs.count > compact_at) filter_compact<NT>(fs, fb, fi, a.K, sc);
+      // every thread reads the count before anyone offers again: one decision
+      const int cnt = fs.count;
+      group_sync(NT);
+      if (cnt > compact_at) filter_compact<NT>(fs, fb, fi, a.K, sc);
     }
 #pragma unroll
     for (int u = 0; u < kTopkVec; ++u) cur[u] = nxt[u];

@@ -40,9 +40,10 @@ def test_noalloc_matches_topk_select_on_two_calls():
         assert torch.equal(got_i, ref_i)
         assert torch.equal(got_v.view(torch.int32), ref_v.view(torch.int32))
     # beyond the scratch limit: a clear error, nothing launched
-    big = torch.zeros((64, 65536), device="cuda")
-    out = torch.empty((64, 2048), dtype=torch.int32, device="cuda")
-    rc = binding.lib().topk_select_noalloc(big.data_ptr(), None, 64, 65536, 65536, 2048,
+    # (256 rows x 4 chunks x K = 2048 candidates: 2M entries, twice the limit)
+    big = torch.zeros((256, 65536), device="cuda")
+    out = torch.empty((256, 2048), dtype=torch.int32, device="cuda")
+    rc = binding.lib().topk_select_noalloc(big.data_ptr(), None, 256, 65536, 65536, 2048,
                                            out.data_ptr(), None, None)
     assert rc == binding.IDX_ENOWORKSPACE
     ctx.close()
