@@ -88,9 +88,11 @@ IDX_API int idx_destroy(idx_ctx* ctx);
 
 /*
  * Scores only: scores[b][t][p] for every p < N (-inf for p >= len[b]).
- * B*T <= max_rows, N <= max_n.  Decode shapes (T*Q small) run on CUDA cores
- * with the query heads pre-summed in fp32; prefill chunks (T*Q == 128,
- * D == 128) run a tcgen05 tensor-core product with fp32 accumulation in TMEM.
+ * B*T <= max_rows, N <= max_n.  Decode shapes with D in {64, 128} and
+ * T*Q <= 64 run a tcgen05 product (pages x query rows) with fp32 accumulation
+ * in TMEM and the head-sum on the accumulators; other decode shapes run on CUDA
+ * cores with the query heads pre-summed in fp32; prefill chunks (32 <= T*Q <=
+ * 128, Q a power of two, D == 128) run a tcgen05 product of query rows x pages.
  * The fp32 result is within 1e-5 * sum_h sum_d |q_hd * c_pd| of the exact score.
  */
 IDX_API int centroid_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths,
@@ -117,6 +119,28 @@ IDX_API int topk_select(idx_ctx* ctx, const float* scores, const int32_t* length
 IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths,
                      int B, int T, int Q, int D, int N, int64_t ldc_b, int K, int32_t* idx_out,
                      float* val_out, idx_stream stream);
+
+/*
+ * Multi-token decode with a valid page count per token row: token t of
+ * request b sees pages p < token_lengths[b*T + t] (device int32 [B*T], each
+ * in [0, N]); every other page of its row is -inf and never selected.  In
+ * causal decoding of T new tokens after pos0[b] tokens of context, with pages
+ * of P keys, token t sees ceil((pos0[b] + t + 1) / P) pages: the per-token
+ * "dead" tail of a multi-token chunk ("Round 15 Track C Audit", section 1
+ * Target 1 item 3; the pos0 x ntok grid of "Round 18 Track C", section 2).
+ * Each request streams the pages of its longest row once for all its tokens.
+ * Otherwise as centroid_score / score_topk_fused (the prefill tensor-core
+ * route is not used: those shapes go through the decode kernels), with the
+ * same limits and errors; a NULL token_lengths is IDX_EINVAL.  The fused
+ * call's scores are bit-identical to centroid_score_tokens'.
+ */
+IDX_API int centroid_score_tokens(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                                  const int32_t* token_lengths, int B, int T, int Q, int D,
+                                  int N, int64_t ldc_b, float* scores, idx_stream stream);
+IDX_API int score_topk_fused_tokens(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                                    const int32_t* token_lengths, int B, int T, int Q, int D,
+                                    int N, int64_t ldc_b, int K, int32_t* idx_out,
+                                    float* val_out, idx_stream stream);
 
 /*
  * Device-side status of the context: waits for `stream`, reads and clears the

@@ -55,12 +55,13 @@ def _load():
         I = ctypes.c_int
         L = ctypes.c_int64
         lib.oracle_scores.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
+        lib.oracle_scores_tokens.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
         lib.oracle_scores_at.argtypes = [P, P, I, I, I, I, I, L, L, P, P, P, P, P]
         lib.oracle_topk_f64.argtypes = [P, I, I, P, P]
         lib.oracle_topk_f32.argtypes = [P, I, I, P, P]
         lib.oracle_topk_rows_f32.argtypes = [P, P, I, I, L, I, P, P]
         lib.oracle_topk_rows_f64.argtypes = [P, P, I, I, L, I, P, P]
-        for f in ("oracle_scores", "oracle_scores_at", "oracle_topk_f64", "oracle_topk_f32",
+        for f in ("oracle_scores", "oracle_scores_tokens", "oracle_scores_at", "oracle_topk_f64", "oracle_topk_f32",
                   "oracle_topk_rows_f32", "oracle_topk_rows_f64"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -79,17 +80,26 @@ def scores(q_bits, c_bits, lengths=None):
     """Exact scores S and bound scales A, both double [B][T][N].
 
     ``q_bits``: uint16 bf16 patterns [B][T][Q][D]; ``c_bits``: uint16 [B][N][D];
-    ``lengths``: int32 [B] in [0, N] or None (all valid).
+    ``lengths``: int32 [B] in [0, N], int32 [B][T] (a valid page count per
+    token: multi-token causal decode), or None (all valid).
     """
     q = _c(q_bits, np.uint16)
     c = _c(c_bits, np.uint16)
     B, T, Q, D = q.shape
     Bc, N, Dc = c.shape
     assert Bc == B and Dc == D
-    ln = None if lengths is None else _c(lengths, np.int32)
     S = np.empty((B, T, N), np.float64)
     A = np.empty((B, T, N), np.float64)
-    rc = _load().oracle_scores(_ptr(q), _ptr(c), _ptr(ln), B, T, Q, D, N, N * D, _ptr(S), _ptr(A))
+    if lengths is not None and np.ndim(lengths) == 2:
+        # per (request, token) valid page counts: multi-token causal decode
+        ln = _c(lengths, np.int32)
+        assert ln.shape == (B, T)
+        rc = _load().oracle_scores_tokens(_ptr(q), _ptr(c), _ptr(ln), B, T, Q, D, N, N * D,
+                                          _ptr(S), _ptr(A))
+    else:
+        ln = None if lengths is None else _c(lengths, np.int32)
+        rc = _load().oracle_scores(_ptr(q), _ptr(c), _ptr(ln), B, T, Q, D, N, N * D,
+                                   _ptr(S), _ptr(A))
     if rc != 0:
         raise ValueError("oracle_scores: arguments outside the contract")
     return S, A

@@ -104,6 +104,44 @@ ORACLE_API int oracle_scores(const uint16_t* q, const uint16_t* c,
     return 0;
 }
 
+/*
+ * Scores with a valid page count per (request, token): multi-token decode
+ * where token t of request b sees only the pages before its own position
+ * (the per-token "dead" tail of "Round 15 Track C Audit", section 1 Target 1
+ * item 3, and the pos0 x ntok grid of "Round 18 Track C", section 2).
+ *   tok_lengths  [B][T] valid page counts in [0, N]
+ *   S, A         double [B][T][N]; entries p >= tok_lengths[b][t] get
+ *                S = -inf, A = 0
+ */
+ORACLE_API int oracle_scores_tokens(const uint16_t* q, const uint16_t* c,
+                                    const int32_t* tok_lengths, int B, int T,
+                                    int Q, int D, int N, int64_t ldc_b,
+                                    double* S, double* A)
+{
+    if (B < 0 || T < 0 || Q <= 0 || D <= 0 || N < 0 || ldc_b < (int64_t)N * D ||
+        !tok_lengths)
+        return -1;
+    for (int b = 0; b < B; ++b) {
+        for (int t = 0; t < T; ++t) {
+            const int len = tok_lengths[(int64_t)b * T + t];
+            if (len < 0 || len > N) return -1;
+            const uint16_t* q_bt = q + ((int64_t)b * T + t) * Q * D;
+            double* s_row = S + ((int64_t)b * T + t) * N;
+            double* a_row = A + ((int64_t)b * T + t) * N;
+            for (int p = 0; p < N; ++p) {
+                if (p >= len) {
+                    s_row[p] = -INFINITY;
+                    a_row[p] = 0.0;
+                    continue;
+                }
+                score_one(q_bt, c + (int64_t)b * ldc_b + (int64_t)p * D, Q, D,
+                          &s_row[p], &a_row[p]);
+            }
+        }
+    }
+    return 0;
+}
+
 /* Scores at n listed (b, t, p) triples, for spot checks at full size. */
 ORACLE_API int oracle_scores_at(const uint16_t* q, const uint16_t* c, int B,
                                 int T, int Q, int D, int N, int64_t ldc_b,

@@ -32,6 +32,8 @@ SIGNATURES = {
     "centroid_score": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _P, _P]),
     "topk_select": (_I, [_P, _P, _P, _I, _I, _L, _I, _P, _P, _P]),
     "score_topk_fused": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _I, _P, _P, _P]),
+    "centroid_score_tokens": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _P, _P]),
+    "score_topk_fused_tokens": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _I, _P, _P, _P]),
     "idx_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "idx_strerror": (ctypes.c_char_p, [_I]),
     "idx_num_sms": (_I, [_P]),
@@ -177,6 +179,36 @@ def score_topk_fused(ctx, q, c, lengths, K, idx_out, val_out=None, stream=None):
     _check(lib().score_topk_fused(ctx.handle, _ptr(q), _ptr(c), _ptr(lengths), B, T, Q, D, N, ldc,
                                   K, _ptr(idx_out), _ptr(val_out), _stream(stream, q.device)),
            "score_topk_fused")
+    return idx_out, val_out
+
+
+def _token_lengths(token_lengths, B, T):
+    if (tuple(token_lengths.shape) not in ((B, T), (B * T,)) or token_lengths.dtype != torch.int32
+            or not token_lengths.is_contiguous()):
+        raise ValueError("token_lengths must be contiguous int32 [B][T]")
+    return token_lengths
+
+
+def centroid_score_tokens(ctx, q, c, token_lengths, scores, stream=None):
+    """centroid_score with a valid page count per (request, token) row."""
+    B, T, Q, D, N, ldc = _score_shapes(q, c)
+    _token_lengths(token_lengths, B, T)
+    if tuple(scores.shape) != (B, T, N) or scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous fp32 [B][T][N]")
+    _check(lib().centroid_score_tokens(ctx.handle, _ptr(q), _ptr(c), _ptr(token_lengths), B, T, Q,
+                                       D, N, ldc, _ptr(scores), _stream(stream, q.device)),
+           "centroid_score_tokens")
+    return scores
+
+
+def score_topk_fused_tokens(ctx, q, c, token_lengths, K, idx_out, val_out=None, stream=None):
+    """score_topk_fused with a valid page count per (request, token) row."""
+    B, T, Q, D, N, ldc = _score_shapes(q, c)
+    _token_lengths(token_lengths, B, T)
+    _check(lib().score_topk_fused_tokens(ctx.handle, _ptr(q), _ptr(c), _ptr(token_lengths), B, T,
+                                         Q, D, N, ldc, K, _ptr(idx_out), _ptr(val_out),
+                                         _stream(stream, q.device)),
+           "score_topk_fused_tokens")
     return idx_out, val_out
 
 

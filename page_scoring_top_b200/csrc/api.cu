@@ -99,9 +99,13 @@ int run_topk(idx_ctx* ctx, const float* scores, const int32_t* lengths, int len_
   return status_of(idx::launch_topk(a, stream));
 }
 
-int run_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths, int B,
-              int T, int Q, int D, int N, int64_t ldc_b, float* scores, cudaStream_t stream) {
-  if (idx::prefill_supported(T, Q, D, ldc_b)) {
+// Scores into `scores` [B][T][N].  Per-token page counts (tok_lengths
+// [B*T], lengths unused) always take the decode kernels, which mask each
+// token row; the prefill kernel serves whole-request lengths only.
+int run_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths,
+              const int32_t* tok_lengths, int B, int T, int Q, int D, int N, int64_t ldc_b,
+              float* scores, cudaStream_t stream) {
+  if (!tok_lengths && idx::prefill_supported(T, Q, D, ldc_b)) {
     for (int b0 = 0; b0 < B; b0 += idx::kPrefillMaxB) {
       idx::PrefillArgs p{};
       p.q = q + (int64_t)b0 * T * Q * D;
@@ -125,7 +129,8 @@ int run_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t*
     idx::DecodeArgs a{};
     a.q = q + (int64_t)b0 * T * Q * D;
     a.c = c + (int64_t)b0 * ldc_b;
-    a.lengths = lengths ? lengths + b0 : nullptr;
+    a.lengths = (lengths && !tok_lengths) ? lengths + b0 : nullptr;
+    a.tok_lengths = tok_lengths ? tok_lengths + (int64_t)b0 * T : nullptr;
     a.B = nb;
     a.T = T;
     a.Q = Q;
@@ -232,7 +237,20 @@ IDX_API int centroid_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
   if (!scores || !aligned16(scores)) return IDX_EINVAL;
   DeviceGuard guard(ctx->device);
   if (!guard.ok()) return IDX_ECUDA;
-  return run_score(ctx, q, c, lengths, B, T, Q, D, N, ldc_b, scores, (cudaStream_t)stream);
+  return run_score(ctx, q, c, lengths, nullptr, B, T, Q, D, N, ldc_b, scores,
+                   (cudaStream_t)stream);
+}
+
+IDX_API int centroid_score_tokens(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                                  const int32_t* token_lengths, int B, int T, int Q, int D,
+                                  int N, int64_t ldc_b, float* scores, idx_stream stream) {
+  int rc = check_score_args(ctx, q, c, B, T, Q, D, N, ldc_b);
+  if (rc != IDX_OK) return rc;
+  if (!token_lengths || !scores || !aligned16(scores)) return IDX_EINVAL;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  return run_score(ctx, q, c, nullptr, token_lengths, B, T, Q, D, N, ldc_b, scores,
+                   (cudaStream_t)stream);
 }
 
 IDX_API int topk_select(idx_ctx* ctx, const float* scores, const int32_t* lengths, int rows,
@@ -250,10 +268,12 @@ IDX_API int topk_select(idx_ctx* ctx, const float* scores, const int32_t* length
                   (cudaStream_t)stream);
 }
 
-IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
-                             const int32_t* lengths, int B, int T, int Q, int D, int N,
-                             int64_t ldc_b, int K, int32_t* idx_out, float* val_out,
-                             idx_stream stream) {
+// score_topk_fused with whole-request lengths or, when tok_lengths is set,
+// a valid page count per (request, token) row.
+static int fused_impl(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                      const int32_t* lengths, const int32_t* tok_lengths, int B, int T, int Q,
+                      int D, int N, int64_t ldc_b, int K, int32_t* idx_out, float* val_out,
+                      idx_stream stream) {
   int rc = check_score_args(ctx, q, c, B, T, Q, D, N, ldc_b);
   if (rc != IDX_OK) return rc;
   if (!idx_out) return IDX_EINVAL;
@@ -263,13 +283,14 @@ IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
   if (!guard.ok()) return IDX_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;
   if (T <= idx::kDecodeMaxTFused && K <= idx::decode_fused_max_k(T) &&
-      !idx::prefill_supported(T, Q, D, ldc_b)) {
+      (tok_lengths || !idx::prefill_supported(T, Q, D, ldc_b))) {
     for (int b0 = 0; b0 < B; b0 += idx::kDecodeMaxB) {
       const int nb = std::min(idx::kDecodeMaxB, B - b0);
       idx::DecodeArgs a{};
       a.q = q + (int64_t)b0 * T * Q * D;
       a.c = c + (int64_t)b0 * ldc_b;
-      a.lengths = lengths ? lengths + b0 : nullptr;
+      a.lengths = (lengths && !tok_lengths) ? lengths + b0 : nullptr;
+      a.tok_lengths = tok_lengths ? tok_lengths + (int64_t)b0 * T : nullptr;
       a.B = nb;
       a.T = T;
       a.Q = Q;
@@ -295,9 +316,28 @@ IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
   // Prefill chunks (and token counts beyond the fused CUDA-core path): score
   // into the context's scratch, then select each (request, token) row.
   if ((int64_t)B * T * N > ctx->scratch_elems) return IDX_ENOWORKSPACE;
-  rc = run_score(ctx, q, c, lengths, B, T, Q, D, N, ldc_b, ctx->scratch, st);
+  rc = run_score(ctx, q, c, lengths, tok_lengths, B, T, Q, D, N, ldc_b, ctx->scratch, st);
   if (rc != IDX_OK) return rc;
+  if (tok_lengths)  // one length per row
+    return run_topk(ctx, ctx->scratch, tok_lengths, 1, B * T, N, N, K, idx_out, val_out, st);
   return run_topk(ctx, ctx->scratch, lengths, T, B * T, N, N, K, idx_out, val_out, st);
+}
+
+IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                             const int32_t* lengths, int B, int T, int Q, int D, int N,
+                             int64_t ldc_b, int K, int32_t* idx_out, float* val_out,
+                             idx_stream stream) {
+  return fused_impl(ctx, q, c, lengths, nullptr, B, T, Q, D, N, ldc_b, K, idx_out, val_out,
+                    stream);
+}
+
+IDX_API int score_topk_fused_tokens(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
+                                    const int32_t* token_lengths, int B, int T, int Q, int D,
+                                    int N, int64_t ldc_b, int K, int32_t* idx_out,
+                                    float* val_out, idx_stream stream) {
+  if (!token_lengths) return IDX_EINVAL;
+  return fused_impl(ctx, q, c, nullptr, token_lengths, B, T, Q, D, N, ldc_b, K, idx_out, val_out,
+                    stream);
 }
 
 IDX_API int idx_get_status(idx_ctx* ctx, idx_stream stream, int* bits) {

@@ -308,11 +308,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
 #pragma unroll
             for (int t = 0; t < TT; ++t) {
               if (t0 + t < T) {
+                const int page = p0 + sp + my_page;
+                // per-token counts: a token row ends before the request's longest
+                const bool ok = !a.tok_lengths || page < tok_length(a, b, t0 + t);
                 if (FUSED) {
-                  fused_offer<HIST>(fsel, t0 + t, __float_as_uint(acc[t][0]),
-                                    (uint32_t)(p0 + sp + my_page), mine);
+                  fused_offer<HIST>(fsel, t0 + t, __float_as_uint(acc[t][0]), (uint32_t)page,
+                                    mine && ok);
                 } else if (mine) {
-                  a.scores[((int64_t)b * T + t0 + t) * N + p0 + sp + my_page] = acc[t][0];
+                  a.scores[((int64_t)b * T + t0 + t) * N + page] =
+                      ok ? acc[t][0] : __uint_as_float(kNegInfBits);
                 }
               }
             }

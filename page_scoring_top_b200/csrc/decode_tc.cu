@@ -355,7 +355,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               }
 #pragma unroll
               for (int t = 0; t < TM; ++t)
-                if (t < T) fused_offer<HIST>(fsel, t, __float_as_uint(st[t]), (uint32_t)page, mine);
+                if (t < T) {
+                  // per-token counts: a token row ends before the request's longest
+                  const bool ok = mine && (!a.tok_lengths || page < tok_length(a, b, t));
+                  fused_offer<HIST>(fsel, t, __float_as_uint(st[t]), (uint32_t)page, ok);
+                }
             } else {
               float s = -0.f;
               int h = 0, t = 0;
@@ -364,7 +368,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (col < rows) {
                   s += __uint_as_float(v[col]);
                   if (++h == Q) {
-                    if (mine) a.scores[((int64_t)b * T + t) * N + page] = s;
+                    if (mine)
+                      a.scores[((int64_t)b * T + t) * N + page] =
+                          (!a.tok_lengths || page < tok_length(a, b, t))
+                              ? s
+                              : __uint_as_float(kNegInfBits);
                     s = -0.f;
                     h = 0;
                     ++t;

@@ -227,6 +227,17 @@ __device__ __forceinline__ void score_padding(const DecodeArgs& a, const int* s_
   }
 }
 
+// Valid pages of token t of request b when the call carries per-token
+// counts (clamped to [0, N]; an out-of-range value is reported).
+__device__ __forceinline__ int tok_length(const DecodeArgs& a, int b, int t) {
+  int len = __ldg(a.tok_lengths + (int64_t)b * a.T + t);
+  if (len < 0 || len > a.N) {
+    if (blockIdx.x == 0) atomicOr(a.status, kErrLengthClamped);
+    len = len < 0 ? 0 : a.N;
+  }
+  return len;
+}
+
 // Prefix sums of the clamped request lengths: s_off[b] = first global page of
 // request b, s_off[B] = all valid pages (all nthreads threads; s_wsum holds
 // one word per warp).  A length outside [0, N] is clamped and reported.
@@ -239,10 +250,14 @@ __device__ __forceinline__ void length_prefix(const DecodeArgs& a, int* s_off, u
     const int i = base + tid;
     int len = 0;
     if (i < a.B) {
-      len = a.lengths ? a.lengths[i] : a.N;
-      if (len < 0 || len > a.N) {
-        if (blockIdx.x == 0) atomicOr(a.status, kErrLengthClamped);
-        len = len < 0 ? 0 : a.N;
+      if (a.tok_lengths) {  // a request streams the pages of its longest token row
+        for (int t = 0; t < a.T; ++t) len = max(len, tok_length(a, i, t));
+      } else {
+        len = a.lengths ? a.lengths[i] : a.N;
+        if (len < 0 || len > a.N) {
+          if (blockIdx.x == 0) atomicOr(a.status, kErrLengthClamped);
+          len = len < 0 ? 0 : a.N;
+        }
       }
     }
     const uint32_t incl = warp_incl_scan((uint32_t)len);

@@ -35,7 +35,8 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 struct DecodeArgs {
   const uint16_t* q;
   const uint16_t* c;
-  const int32_t* lengths;  // per request, or null
+  const int32_t* lengths;      // per request, or null
+  const int32_t* tok_lengths;  // per (request, token) [B*T] instead of lengths, or null
   int B, T, Q, D, N;
   int64_t ldc_b;
   int K;

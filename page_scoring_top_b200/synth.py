@@ -150,6 +150,21 @@ def decode_inputs(seed, B, T, Q, D, N, lengths=None, len_range=None, page_bias=F
     return {"q": q, "c": c, "lengths": lengths}
 
 
+def causal_token_lengths(pos0, T, page_tokens, N):
+    """Valid page counts per (request, token) of a multi-token decode step.
+
+    Request b has ``pos0[b]`` tokens of context before this step and decodes
+    T new tokens; token t sits at position pos0[b] + t and sees the keys at
+    positions 0 .. pos0[b] + t, i.e. the first ceil((pos0[b] + t + 1) /
+    page_tokens) pages (capped at N).  This is the per-token "dead" tail of a
+    multi-token chunk, with pages of ``page_tokens`` keys each.  Returns int32
+    [B][T]; the last token's count is the request's page count."""
+    pos0 = np.asarray(pos0, np.int64)
+    t = np.arange(T, dtype=np.int64)
+    n = (pos0[:, None] + t[None, :] + page_tokens) // page_tokens
+    return np.minimum(n, N).astype(np.int32)
+
+
 # --------------------------------------------------------------------------
 # Standalone top-K sweep: fp32 score rows from eleven distributions
 # --------------------------------------------------------------------------

@@ -362,3 +362,47 @@ def test_exact_check_rejects_planted_score_mistakes():
         assert not ok, name
     for p in range(5):
         assert abs(Fraction(S[0, 0, p]) - exact[0, p]) <= Fraction(12) * Fraction(2.0 ** -53) * Fraction(A[0, 0, p])
+
+
+# ------------------------------------------------------------------ per-token (multi-token decode) rows
+
+def test_causal_token_lengths_worked_example():
+    # pages of 4 keys; context 5 tokens, 4 new tokens at positions 5, 6, 7, 8:
+    # they see 6, 7, 8, 9 keys -> 2, 2, 2, 3 pages.  Context 0: 1..4 keys -> 1 page.
+    # Context 7: 8 keys -> 2 pages, then 9, 10, 11 keys -> 3 pages.  Capped at N.
+    got = synth.causal_token_lengths([5, 0, 7, 100], 4, 4, 26)
+    want = [[2, 2, 2, 3], [1, 1, 1, 1], [2, 3, 3, 3], [26, 26, 26, 26]]
+    assert got.tolist() == want
+
+
+def test_token_lengths_scores_by_hand():
+    # Q=1, D=2, q_t = [t+1, 0]: token t's score of page p is (t+1) * c[p,0];
+    # token 0 sees 1 page, token 1 sees 3 pages.
+    q = _bf16([[[[1.0, 0.0]], [[2.0, 0.0]]]])          # [1][2][1][2]
+    c = _bf16([[[1.0, 5.0], [3.0, -1.0], [-2.0, 4.0]]])  # [1][3][2]
+    S, A = oracle.scores(q, c, np.array([[1, 3]], np.int32))
+    assert S[0, 0].tolist() == [1.0, -np.inf, -np.inf]
+    assert S[0, 1].tolist() == [2.0, 6.0, -4.0]
+    assert A[0, 0].tolist() == [1.0, 0.0, 0.0]
+    idx, val, kk = oracle.topk(S[0, 1], 2)
+    assert idx.tolist() == [1, 0] and kk == 2
+
+
+@pytest.mark.parametrize("seed", [21, 22])
+def test_token_lengths_equal_masked_request_rows(seed):
+    # a token row is its request row with the pages past the token's count at -inf
+    B, T, N = 3, 4, 40
+    d = synth.decode_inputs(seed, B=B, T=T, Q=2, D=16, N=N, lengths=[N, 30, 0])
+    tl = synth.causal_token_lengths([150, 113, 0], T, 4, N)
+    tl[2] = 0
+    S_req, A_req = oracle.scores(d["q"], d["c"], tl[:, -1])
+    S_tok, A_tok = oracle.scores(d["q"], d["c"], tl)
+    live = np.arange(N)[None, None, :] < tl[:, :, None]
+    assert np.array_equal(S_tok, np.where(live, S_req, -np.inf))
+    assert np.array_equal(A_tok, np.where(live, A_req, 0.0))
+    # and the per-row select sees exactly the live pages
+    idx, _ = oracle.topk_rows(S_tok.reshape(B * T, N), 8, tl.reshape(-1))
+    for r in range(B * T):
+        sel = idx[r][idx[r] >= 0]
+        assert np.all(sel < tl.reshape(-1)[r])
+        assert len(sel) == min(8, tl.reshape(-1)[r])
