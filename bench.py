@@ -10,12 +10,14 @@ request are written.  The metric is valid pages scored+selected per second
 (whole job) and the HBM bandwidth that implies.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                       [--workload ragged_decode|prefill_chunk|batch_decode_bias|tiny_decode]
+                       [--workload ragged_decode|prefill_chunk|causal_decode|...]
 
 The default workload is the headline one above.  The others are the indexer's
 remaining workloads, for profiling: a prefill chunk (B=4, T=16, Q=8, N=131072,
 K=512; every token row of 131072 pages selects its top 512) counts one unit per
-(token row, page).
+(token row, page); a multi-token causal decode step (B=32 requests, 4 new
+tokens each, per-token page counts, K=256) counts one unit per (token row,
+valid page of that row).
 For N > 1 launch under torch.distributed.run: requests are sharded across ranks
 (each rank owns its batch; no collective on the data path), timing is the max
 over ranks.  ``--impl reference`` times the CPU oracle (single-threaded C) on
@@ -64,7 +66,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=("ragged_decode", "prefill_chunk", "batch_decode_bias", "tiny_decode"))
+                    choices=("ragged_decode", "prefill_chunk", "causal_decode",
+                             "batch_decode_bias", "tiny_decode"))
     return ap.parse_args()
 
 
@@ -249,16 +252,23 @@ def run_ours(args):
     K = spec["K"]
     pages, nbytes = algorithmic_bytes(d["lengths"], B, T, Q, D, K, with_values=False)
     units = pages * T  # (token row, valid page) pairs scored and selected
+    tok = d.get("token_lengths")
+    if tok is not None:
+        units = int(np.sum(tok))
 
     q = torch.from_numpy(d["q"].view(np.int16)).to(dev)
     c = torch.from_numpy(d["c"].view(np.int16)).to(dev)
     ln = torch.from_numpy(d["lengths"]).to(dev)
+    tokd = None if tok is None else torch.from_numpy(np.ascontiguousarray(tok)).to(dev)
     idx = torch.empty((B * T, K), dtype=torch.int32, device=dev)
     ctx = binding.Context(local, max_rows=B * T, max_n=N, max_k=K)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        binding.score_topk_fused(ctx, q, c, ln, K, idx, None, stream=stream)
+        if tokd is not None:
+            binding.score_topk_fused_tokens(ctx, q, c, tokd, K, idx, None, stream=stream)
+        else:
+            binding.score_topk_fused(ctx, q, c, ln, K, idx, None, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -306,7 +316,9 @@ def run_ours(args):
     launch_s = (ms / args.steps) * 1e-3
     score_bytes = nbytes
     tensor = None
-    if T > 1:
+    if tok is not None:
+        kernel = "decode_tc_kernel<D=128,NC=16,fused> (4 token rows per request)"
+    elif T > 1:
         kernel = PREFILL_KERNEL
         scores = torch.empty((B, T, N), dtype=torch.float32, device=dev)
         for _ in range(args.warmup):
@@ -343,6 +355,8 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": args.workload, "B": B, "T": T, "Q": Q, "D": D, "N": N, "K": K,
                        "len_dist": ("uniform 1024..65536" if args.workload == WORKLOAD
+                                    else "causal: context U{64*1024..64*65536-4} keys, "
+                                         "64 keys per page" if tok is not None
                                     else "all pages valid"), "seed": seed,
                        "pages_per_step_per_gpu": pages, "bytes_per_step_per_gpu": nbytes,
                        "parallelism": "dp%d (requests sharded, no data-path collective)" % world,
@@ -352,7 +366,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                          "kernel": kernel},
-            "gpu_launches": args.steps * (2 if T > 1 else 1),
+            "gpu_launches": args.steps * (2 if (T > 1 and tok is None) else 1),
             "clocks": clocks,
             "tensor": tensor,
             "e2e": e2e,

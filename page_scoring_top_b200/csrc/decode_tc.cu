@@ -304,7 +304,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // check that leaves `room` free entries the next one comes within
     // room / 128 tiles.  With the histogram the compaction is only the
     // overflow guard; without it, it also raises the threshold.
-    const int compact_at = FUSED ? (HIST ? L.cap - 2 * kTcTile : fused_compact_at<HIST>(L.cap, a.K)) : 0;
+    // (without it, a filter compacts once it holds twice K entries -- the
+    // threshold then tracks the K-th value -- and always before the room
+    // runs out; small per-token filters would otherwise compact every check)
+    const int compact_at =
+        FUSED ? (HIST ? L.cap - 2 * kTcTile
+                      : max(fused_compact_at<HIST>(L.cap, a.K), min(L.cap - 2 * kTcTile, 2 * a.K)))
+              : 0;
     uint32_t tile = 0;
     for (int j = g; j < nchunks; j += G) {
       const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);

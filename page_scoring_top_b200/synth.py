@@ -246,6 +246,11 @@ WORKLOADS = {
     "ragged_decode": dict(seed=103, B=32, T=1, Q=4, D=128, N=65536, K=256,
                           len_range=(1024, 65536)),
     "prefill_chunk": dict(seed=105, B=4, T=16, Q=8, D=128, N=131072, K=512),
+    # multi-token causal decode: 4 new tokens after a ragged context of
+    # U{64*1024 .. 64*65536 - 4} keys, pages of 64 keys (token lengths drawn
+    # from stream 4 of the seed)
+    "causal_decode": dict(seed=106, B=32, T=4, Q=4, D=128, N=65536, K=256,
+                          pos0_range=(64 * 1024, 64 * 65536 - 4), page_tokens=64),
 }
 SWEEP_SEED = 104
 
@@ -255,6 +260,17 @@ def workload(name, **override):
     spec = dict(WORKLOADS[name])
     spec.update(override)
     K = spec.pop("K")
+    if "pos0_range" in spec:
+        lo, hi = spec.pop("pos0_range")
+        page_tokens = spec.pop("page_tokens")
+        u = uniform53(u64(spec["seed"], 4, 0, spec["B"]))
+        pos0 = lo + np.floor(u * (hi - lo + 1)).astype(np.int64)
+        tl = causal_token_lengths(pos0, spec["T"], page_tokens, spec["N"])
+        inputs = decode_inputs(spec.pop("seed"), spec.pop("B"), spec.pop("T"), spec.pop("Q"),
+                               spec.pop("D"), spec.pop("N"), lengths=tl[:, -1], **spec)
+        inputs["token_lengths"] = tl
+        inputs["K"] = K
+        return inputs
     inputs = decode_inputs(spec.pop("seed"), spec.pop("B"), spec.pop("T"), spec.pop("Q"),
                            spec.pop("D"), spec.pop("N"), **spec)
     inputs["K"] = K
