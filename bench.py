@@ -52,7 +52,7 @@ FALLBACK_HBM_GBS = 6650.0
 # summarised in profiles/decode_fused_ragged_decode.md: (301.28 MB read +
 # 3.95 MB written) per launch / 1,175,731 pages.  Set to None whenever the
 # kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES_PER_PAGE = 259.6
+NCU_TRAFFIC_BYTES_PER_PAGE = None  # kernel changed since the 259.6 B/page capture
 
 
 def parse():

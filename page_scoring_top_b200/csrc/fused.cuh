@@ -22,7 +22,7 @@ constexpr int kMaxFusedT = 4;
 // Virtual pages charged per request in fused mode: about what a segment-end
 // select step costs in streaming time (a few microseconds at one SM's share
 // of HBM bandwidth, minus what the stage ring absorbs).
-constexpr int kSegmentPages = 512;
+constexpr int kSegmentPages = 896;
 
 // Shared-memory state of the fused select (pointers into the kernel's layout).
 struct FusedSel {
