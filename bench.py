@@ -66,7 +66,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=("ragged_decode", "prefill_chunk", "causal_decode",
+                    choices=("ragged_decode", "prefill_chunk", "causal_decode", "pool_keys",
                              "batch_decode_bias", "tiny_decode"))
     return ap.parse_args()
 
@@ -428,10 +428,70 @@ def measure_e2e(binding, ctx, d, K, dev, stream, steps, barrier, pg):
             "steps": steps, "ms_per_step": ms_max / steps}
 
 
+def run_pool(args):
+    """Page centroids by key mean-pooling (the producer of the centroid
+    table): 4 requests x 131072 keys of D=128 in pages of 64, one
+    centroid_pool call per step; units are pages pooled."""
+    import torch
+    from page_scoring_top_b200 import binding, synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B, P, N, D = 4, 64, 2048, 128
+    keys = synth.normal_bf16(107, 1, 0, B * N * P * D).reshape(B, N * P, D)
+    counts = np.full(B, N * P, np.int32)
+    kd = torch.from_numpy(keys.view(np.int16)).to(dev)
+    kc = torch.from_numpy(counts).to(dev)
+    cd = torch.empty((B, N, D), dtype=torch.int16, device=dev)
+    ctx = binding.Context(0, max_rows=B, max_n=N, max_k=1)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        binding.centroid_pool(ctx, kd, kc, P, cd, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.15)
+    e0.record(stream)
+    for _ in range(args.steps):
+        binding.centroid_pool(ctx, kd, kc, P, cd, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    rc, bits = binding.idx_get_status(ctx)
+    if rc != 0:
+        raise RuntimeError("device status %d" % bits)
+    pages = B * N
+    nbytes = B * N * P * D * 2 + B * N * D * 2 + B * 4
+    launch_s = ms / args.steps * 1e-3
+    achieved = nbytes / launch_s / 1e9
+    peak, peak_src = measured_peak()
+    line = {
+        "metric": "pages pooled/sec (key mean-pooling into centroids)", "value": pages / launch_s,
+        "unit": "pages/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
+        "config": {"workload": "pool_keys", "B": B, "keys_per_page": P, "pages": N, "D": D,
+                   "bytes_per_step": nbytes,
+                   "l2": "inputs larger than L2 (%.1f MB of keys per step); no flush" %
+                         (B * N * P * D * 2 / 1e6)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                     "kernel": "pool_kernel"},
+        "gpu_launches": args.steps, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    ctx.close()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "pool_keys":
+        return run_pool(args)
     return run_ours(args)
 
 

@@ -143,6 +143,22 @@ IDX_API int score_topk_fused_tokens(idx_ctx* ctx, const uint16_t* q, const uint1
                                     float* val_out, idx_stream stream);
 
 /*
+ * Page centroids by key mean-pooling, the producer of the centroid table the
+ * calls above read (the "pooled keys" of "Round 15 Track C Audit", section 2):
+ *     c[b,p,d] = bf16_rne( (1/n) * sum_{i<n} keys[b, p*P + i, d] ),
+ *     n = min(P, key_counts[b] - p*P)
+ * summed in fp32 and rounded once.  keys: bf16 [B][L][D] with request stride
+ * ldk_b elements (L = ldk_b / D keys of room); key_counts: device int32 [B],
+ * each in [0, min(N*P, L)] (clamped and reported like lengths); c: bf16
+ * [B][N][D] with request stride ldc_b >= N*D.  Pages without a valid key are
+ * not written.  keys and c 16-byte aligned, ldk_b and ldc_b multiples of 8,
+ * D % 8 == 0 and D <= 256.  No workspace is used.
+ */
+IDX_API int centroid_pool(idx_ctx* ctx, const uint16_t* keys, const int32_t* key_counts, int B,
+                          int D, int P, int N, int64_t ldk_b, uint16_t* c, int64_t ldc_b,
+                          idx_stream stream);
+
+/*
  * Device-side status of the context: waits for `stream`, reads and clears the
  * status word.  Returns IDX_OK, or IDX_EDEVICE with *bits (if non-NULL) set to
  * the raised bits: 1 = a length outside [0, N] was clamped, 2 = a bounded wait

@@ -56,12 +56,13 @@ def _load():
         L = ctypes.c_int64
         lib.oracle_scores.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
         lib.oracle_scores_tokens.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
+        lib.oracle_pool.argtypes = [P, P, I, I, I, I, L, P]
         lib.oracle_scores_at.argtypes = [P, P, I, I, I, I, I, L, L, P, P, P, P, P]
         lib.oracle_topk_f64.argtypes = [P, I, I, P, P]
         lib.oracle_topk_f32.argtypes = [P, I, I, P, P]
         lib.oracle_topk_rows_f32.argtypes = [P, P, I, I, L, I, P, P]
         lib.oracle_topk_rows_f64.argtypes = [P, P, I, I, L, I, P, P]
-        for f in ("oracle_scores", "oracle_scores_tokens", "oracle_scores_at", "oracle_topk_f64", "oracle_topk_f32",
+        for f in ("oracle_scores", "oracle_scores_tokens", "oracle_pool", "oracle_scores_at", "oracle_topk_f64", "oracle_topk_f32",
                   "oracle_topk_rows_f32", "oracle_topk_rows_f64"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -103,6 +104,20 @@ def scores(q_bits, c_bits, lengths=None):
     if rc != 0:
         raise ValueError("oracle_scores: arguments outside the contract")
     return S, A
+
+
+def pool(key_bits, key_counts, P, N):
+    """Exact page centroids (double [B][N][D]): the mean of each page's valid
+    keys; ``key_bits`` uint16 bf16 [B][L][D], ``key_counts`` int32 [B] (<= L,
+    <= N*P), pages of P keys."""
+    k = _c(key_bits, np.uint16)
+    B, L, D = k.shape
+    kc = _c(key_counts, np.int32)
+    means = np.empty((B, N, D), np.float64)
+    rc = _load().oracle_pool(_ptr(k), _ptr(kc), B, D, P, N, L * D, _ptr(means))
+    if rc != 0:
+        raise ValueError("oracle_pool: arguments outside the contract")
+    return means
 
 
 def scores_at(q_bits, c_bits, b, t, p):

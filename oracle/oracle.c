@@ -261,3 +261,34 @@ ORACLE_API int oracle_topk_rows_f64(const double* scores, const int32_t* lengths
     }
     return 0;
 }
+
+/*
+ * Page centroids by key mean-pooling (the "pooled keys" that feed the
+ * indexer, "Round 15 Track C Audit", section 2 parity list): request b holds
+ * key_counts[b] keys of D bf16 values at keys + b*ldk_b + i*D; page p covers
+ * keys p*P .. p*P + P - 1, and its centroid is the mean of the page's valid
+ * keys, n = min(P, key_counts[b] - p*P), computed exactly in double.
+ *   means  double [B][N][D]; pages with no valid key get 0
+ * Returns -1 on arguments outside the contract.
+ */
+ORACLE_API int oracle_pool(const uint16_t* keys, const int32_t* key_counts, int B, int D, int P,
+                           int N, int64_t ldk_b, double* means)
+{
+    if (B < 0 || D <= 0 || P <= 0 || N < 0 || !key_counts) return -1;
+    for (int b = 0; b < B; ++b) {
+        const int nk = key_counts[b];
+        if (nk < 0 || (int64_t)nk > (int64_t)N * P || ldk_b < (int64_t)nk * D) return -1;
+        for (int p = 0; p < N; ++p) {
+            double* m = means + ((int64_t)b * N + p) * D;
+            int n = nk - p * P;
+            n = n < 0 ? 0 : (n > P ? P : n);
+            for (int d = 0; d < D; ++d) {
+                double s = 0.0;
+                for (int i = 0; i < n; ++i)
+                    s += bf16_bits_to_double(keys[(int64_t)b * ldk_b + ((int64_t)p * P + i) * D + d]);
+                m[d] = n ? s / n : 0.0;
+            }
+        }
+    }
+    return 0;
+}

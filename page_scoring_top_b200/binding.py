@@ -34,6 +34,7 @@ SIGNATURES = {
     "score_topk_fused": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _I, _P, _P, _P]),
     "centroid_score_tokens": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _P, _P]),
     "score_topk_fused_tokens": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _I, _P, _P, _P]),
+    "centroid_pool": (_I, [_P, _P, _P, _I, _I, _I, _I, _L, _P, _L, _P]),
     "idx_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "idx_strerror": (ctypes.c_char_p, [_I]),
     "idx_num_sms": (_I, [_P]),
@@ -218,3 +219,20 @@ def idx_get_status(ctx, stream=None):
     rc = lib().idx_get_status(ctx.handle, _stream(stream, torch.device("cuda", ctx.device)),
                               ctypes.byref(bits))
     return rc, bits.value
+
+
+def centroid_pool(ctx, keys, key_counts, P, c, stream=None):
+    """c[b,p,:] = bf16 mean of the valid keys of page p (P keys per page).
+    keys: bf16 bits (int16) [B][L][D]; key_counts: int32 [B]; c: int16 [B][N][D]."""
+    if keys.dim() != 3 or keys.dtype != torch.int16 or not keys.is_contiguous():
+        raise ValueError("keys must be contiguous bf16 bits (int16) [B][L][D]")
+    B, Lk, D = keys.shape
+    if c.dim() != 3 or c.dtype != torch.int16 or not c.is_contiguous() or c.shape[0] != B \
+            or c.shape[2] != D:
+        raise ValueError("c must be contiguous bf16 bits (int16) [B][N][D]")
+    N = c.shape[1]
+    if tuple(key_counts.shape) != (B,) or key_counts.dtype != torch.int32:
+        raise ValueError("key_counts must be int32 [B]")
+    _check(lib().centroid_pool(ctx.handle, _ptr(keys), _ptr(key_counts), B, D, P, N, Lk * D,
+                               _ptr(c), N * D, _stream(stream, keys.device)), "centroid_pool")
+    return c

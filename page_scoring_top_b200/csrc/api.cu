@@ -323,6 +323,31 @@ static int fused_impl(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
   return run_topk(ctx, ctx->scratch, lengths, T, B * T, N, N, K, idx_out, val_out, st);
 }
 
+IDX_API int centroid_pool(idx_ctx* ctx, const uint16_t* keys, const int32_t* key_counts, int B,
+                          int D, int P, int N, int64_t ldk_b, uint16_t* c, int64_t ldc_b,
+                          idx_stream stream) {
+  if (!ctx || !keys || !key_counts || !c) return IDX_EINVAL;
+  if (B <= 0 || D <= 0 || P <= 0 || N <= 0) return IDX_EINVAL;
+  if (!aligned16(keys) || !aligned16(c) || (ldk_b % 8) != 0 || (ldc_b % 8) != 0) return IDX_EINVAL;
+  if (ldc_b < (int64_t)N * D || ldk_b < D) return IDX_EINVAL;
+  if ((D % 8) != 0 || D > 256) return IDX_EUNSUPPORTED;
+  if ((int64_t)N * P > INT32_MAX || (int64_t)B * N > INT32_MAX) return IDX_EUNSUPPORTED;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  idx::PoolArgs a{};
+  a.keys = keys;
+  a.key_counts = key_counts;
+  a.B = B;
+  a.D = D;
+  a.P = P;
+  a.N = N;
+  a.ldk_b = ldk_b;
+  a.ldc_b = ldc_b;
+  a.c = c;
+  a.status = ctx->status;
+  return status_of(idx::launch_pool(a, ctx->num_sms, (cudaStream_t)stream));
+}
+
 IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
                              const int32_t* lengths, int B, int T, int Q, int D, int N,
                              int64_t ldc_b, int K, int32_t* idx_out, float* val_out,

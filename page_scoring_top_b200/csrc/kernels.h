@@ -77,4 +77,15 @@ constexpr int kPrefillMaxB = 256;  // requests per launch (host splits larger ba
 bool prefill_supported(int T, int Q, int D, int64_t ldc_b);
 cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t stream);
 
+// ---------------------------------------------------------------- page centroids
+struct PoolArgs {
+  const uint16_t* keys;        // bf16, key i of request b at keys + b*ldk_b + i*D
+  const int32_t* key_counts;   // [B] valid keys per request
+  int B, D, P, N;              // P keys per page, N pages per request
+  int64_t ldk_b, ldc_b;
+  uint16_t* c;                 // bf16 [B][N][D] with request stride ldc_b
+  int* status;
+};
+cudaError_t launch_pool(const PoolArgs& a, int num_sms, cudaStream_t stream);
+
 }  // namespace idx

@@ -406,3 +406,32 @@ def test_token_lengths_equal_masked_request_rows(seed):
         sel = idx[r][idx[r] >= 0]
         assert np.all(sel < tl.reshape(-1)[r])
         assert len(sel) == min(8, tl.reshape(-1)[r])
+
+
+# ------------------------------------------------------------------ page centroids (key mean-pooling)
+
+def test_pool_worked_example():
+    # pages of 2 keys over 5 keys: (1,2)+(3,4) -> (2,3); (5,6)+(7,8) -> (6,7);
+    # the partial last page holds (9,10) alone; page 3 has no key -> 0
+    k = _bf16([[[1, 2], [3, 4], [5, 6], [7, 8], [9, 10]]])
+    m = oracle.pool(k, np.array([5], np.int32), 2, 4)
+    assert m[0].tolist() == [[2, 3], [6, 7], [9, 10], [0, 0]]
+
+
+def test_pool_closed_forms():
+    rng = np.random.default_rng(31)
+    k = synth.normal_bf16(32, 1, 0, 2 * 40 * 8).reshape(2, 40, 8)
+    counts = np.array([40, 23], np.int32)
+    # one key per page: the centroid is the key itself
+    m1 = oracle.pool(k, counts, 1, 40)
+    kf = synth.bf16_bits_to_f32(k).astype(np.float64)
+    assert np.array_equal(m1[0], kf[0]) and np.array_equal(m1[1, :23], kf[1, :23])
+    # constant keys: the centroid is the constant, whatever the page size
+    c = np.full((1, 12, 8), synth.f32_to_bf16_bits(np.array([0.375], np.float32))[0], np.uint16)
+    assert np.all(oracle.pool(c, np.array([12], np.int32), 5, 3) == 0.375)
+    # the mean is linear: pooling 2*k (exact in bf16) doubles it
+    k2 = synth.f32_to_bf16_bits((2 * synth.bf16_bits_to_f32(k)).astype(np.float32))
+    assert np.array_equal(oracle.pool(k2, counts, 4, 10), 2 * oracle.pool(k, counts, 4, 10))
+    # a library mean over the same keys
+    lib = kf[1, 20:23].mean(axis=0)
+    assert np.allclose(oracle.pool(k, counts, 4, 10)[1, 5], lib, rtol=0, atol=1e-15)
