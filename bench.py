@@ -49,10 +49,10 @@ KERNEL = "decode_tc_kernel<D=128,NC=16,fused,hist>"
 PREFILL_KERNEL = "prefill_kernel<Q=8> (tcgen05 score of a 16-token chunk)"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes per valid page of the fused decode kernel, from the ncu capture
-# summarised in profiles/decode_fused_ragged_decode.md: (301.28 MB read +
-# 3.95 MB written) per launch / 1,175,731 pages.  Set to None whenever the
+# summarised in profiles/decode_fused_ragged_decode.md: (301.27 MB read +
+# 3.47 MB written) per launch / 1,175,731 pages.  Set to None whenever the
 # kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES_PER_PAGE = None  # kernel changed since the 259.6 B/page capture
+NCU_TRAFFIC_BYTES_PER_PAGE = 259.2
 
 
 def parse():
