@@ -1,5 +1,9 @@
 // decode.cu -- page scoring on CUDA cores, alone or fused with the top-K select.
 //
+// The decode shapes the tensor-core kernel (decode_tc.cu) does not take --
+// D = 256 or not a multiple of 64, more than 64 query rows -- run here; both
+// kernels share the work split and the select steps (fused.cuh).
+//
 // What is computed ("Iterate Centroids Score", opening description;
 // "Round 18 Track C", section 1 Target 2, qsa_score):
 //     s[b,t,p] = sum_h sum_d q[b,t,h,d] * c[b,p,d]   for p < len[b]
@@ -11,10 +15,11 @@
 //
 // Work decomposition (B200: 148 SMs, one persistent CTA per SM):
 //  * The valid pages of all requests are laid end to end (prefix sums of the
-//    ragged lengths, computed in every CTA) and cut into equal chunks, so a
-//    CTA's load is balanced to within one page however ragged the batch is;
-//    padded pages are never read.
-//  * Warp 8 is the producer: one lane streams 32-page stages of the centroid
+//    ragged lengths, computed in every CTA; in fused mode each request is also
+//    charged a fixed number of virtual pages for its segment-end select) and
+//    cut into equal chunks, so a CTA's load is balanced however ragged the
+//    batch is; padded pages are never read.
+//  * Warp 8 is the producer: four lanes stream 32-page stages of the centroid
 //    table into a shared-memory ring with 1-D bulk copies (TMA engine), an
 //    mbarrier pair per slot, L2 evict-first.
 //  * Warps 0..7 consume stages round-robin.  Four lanes share a page (8 pages
@@ -24,11 +29,13 @@
 //    lane keeps its pre-summed query chunks in registers; a two-step butterfly
 //    of shuffles leaves each lane with one page's full score.
 //  * Score mode writes the scores (and -inf padding) to HBM.  Fused mode offers
-//    each score to an exact online top-K filter in shared memory (select.cuh);
-//    at the end of a row's part of the chunk the filter is compacted to K
-//    candidates, published, and the last CTA to finish the row merges all of
-//    the row's candidates and writes the final indices.  The score row never
-//    reaches HBM and the producer keeps prefetching through every compaction.
+//    each score to an exact online top-K filter in shared memory (fused.cuh:
+//    the digit-histogram filter of hsel.cuh for single-token rows, radix
+//    compaction filters per token otherwise); at the end of a row's part of
+//    the chunk the filter's exact top K is published, and the last CTA to
+//    finish the row merges the row's candidates and writes the final indices.
+//    The score row never reaches HBM and the producer keeps prefetching
+//    through every select step.
 // Both modes run the same arithmetic, so fused and score-mode scores are
 // bit-identical.
 #include "common.cuh"
