@@ -143,6 +143,26 @@ IDX_API int score_topk_fused_tokens(idx_ctx* ctx, const uint16_t* q, const uint1
                                     float* val_out, idx_stream stream);
 
 /*
+ * Paged centroid table: the centroids live in one shared block pool
+ * (bf16 [n_blocks][D], 16-byte aligned) and page p of request b is pool row
+ * page_table[b*ld_pt + p] (device int32, ld_pt >= N; entries past lengths[b]
+ * are not read; an entry outside [0, n_blocks) is clamped and reported as
+ * status bit 4).  This is the block-pool layout of "Iterate Centroids Score"
+ * (the ctx argument indexes each request's pages in a shared table).
+ * Otherwise as centroid_score / score_topk_fused, with the same limits and
+ * errors (pages are gathered row by row on the CUDA-core decode kernel; the
+ * fused call's scores are bit-identical to centroid_score_paged's).
+ */
+IDX_API int centroid_score_paged(idx_ctx* ctx, const uint16_t* q, const uint16_t* pool,
+                                 int n_blocks, const int32_t* page_table, int64_t ld_pt,
+                                 const int32_t* lengths, int B, int T, int Q, int D, int N,
+                                 float* scores, idx_stream stream);
+IDX_API int score_topk_fused_paged(idx_ctx* ctx, const uint16_t* q, const uint16_t* pool,
+                                   int n_blocks, const int32_t* page_table, int64_t ld_pt,
+                                   const int32_t* lengths, int B, int T, int Q, int D, int N,
+                                   int K, int32_t* idx_out, float* val_out, idx_stream stream);
+
+/*
  * Page centroids by key mean-pooling, the producer of the centroid table the
  * calls above read (the "pooled keys" of "Round 15 Track C Audit", section 2):
  *     c[b,p,d] = bf16_rne( (1/n) * sum_{i<n} keys[b, p*P + i, d] ),
@@ -162,7 +182,8 @@ IDX_API int centroid_pool(idx_ctx* ctx, const uint16_t* keys, const int32_t* key
  * Device-side status of the context: waits for `stream`, reads and clears the
  * status word.  Returns IDX_OK, or IDX_EDEVICE with *bits (if non-NULL) set to
  * the raised bits: 1 = a length outside [0, N] was clamped, 2 = a bounded wait
- * inside a kernel expired (that call's output is not valid).  Synchronises.
+ * inside a kernel expired (that call's output is not valid), 4 = a page-table
+ * entry outside the block pool was clamped.  Synchronises.
  */
 IDX_API int idx_get_status(idx_ctx* ctx, idx_stream stream, int* bits);
 

@@ -120,6 +120,20 @@ def pool(key_bits, key_counts, P, N):
     return means
 
 
+def scores_paged(q_bits, pool_bits, page_table, lengths=None):
+    """Scores when page p of request b is row page_table[b, p] of a shared
+    block pool (the block-pool table of "Iterate Centroids Score"): the
+    gather is a library fancy index, the arithmetic is ``scores``'s."""
+    pool = _c(pool_bits, np.uint16)
+    pt = np.asarray(page_table)
+    B, N = pt.shape
+    gathered = pool[np.clip(pt, 0, pool.shape[0] - 1)]  # [B][N][D]
+    if lengths is not None:
+        live = np.arange(N)[None, :] < np.asarray(lengths)[:, None]
+        gathered = np.where(live[:, :, None], gathered, np.uint16(0))
+    return scores(q_bits, gathered, lengths)
+
+
 def scores_at(q_bits, c_bits, b, t, p):
     """Exact S and A at the listed (b, t, p) triples (spot checks at full size)."""
     q = _c(q_bits, np.uint16)

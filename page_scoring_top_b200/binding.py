@@ -35,6 +35,9 @@ SIGNATURES = {
     "centroid_score_tokens": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _P, _P]),
     "score_topk_fused_tokens": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _L, _I, _P, _P, _P]),
     "centroid_pool": (_I, [_P, _P, _P, _I, _I, _I, _I, _L, _P, _L, _P]),
+    "centroid_score_paged": (_I, [_P, _P, _P, _I, _P, _L, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "score_topk_fused_paged": (_I, [_P, _P, _P, _I, _P, _L, _P, _I, _I, _I, _I, _I, _I, _P, _P,
+                                    _P]),
     "idx_get_status": (_I, [_P, _P, ctypes.POINTER(_I)]),
     "idx_strerror": (ctypes.c_char_p, [_I]),
     "idx_num_sms": (_I, [_P]),
@@ -236,3 +239,38 @@ def centroid_pool(ctx, keys, key_counts, P, c, stream=None):
     _check(lib().centroid_pool(ctx.handle, _ptr(keys), _ptr(key_counts), B, D, P, N, Lk * D,
                                _ptr(c), N * D, _stream(stream, keys.device)), "centroid_pool")
     return c
+
+
+def _paged_shapes(q, pool, page_table):
+    if q.dim() != 4 or q.dtype != torch.int16 or not q.is_contiguous():
+        raise ValueError("q must be contiguous bf16 bits (int16) [B][T][Q][D]")
+    if pool.dim() != 2 or pool.dtype != torch.int16 or not pool.is_contiguous():
+        raise ValueError("pool must be contiguous bf16 bits (int16) [n_blocks][D]")
+    if page_table.dim() != 2 or page_table.dtype != torch.int32 or not page_table.is_contiguous():
+        raise ValueError("page_table must be contiguous int32 [B][N]")
+    B, T, Q, D = q.shape
+    if pool.shape[1] != D or page_table.shape[0] != B:
+        raise ValueError("shape mismatch")
+    return B, T, Q, D, page_table.shape[1], pool.shape[0]
+
+
+def centroid_score_paged(ctx, q, pool, page_table, lengths, scores, stream=None):
+    """centroid_score with page p of request b read from pool[page_table[b, p]]."""
+    B, T, Q, D, N, nb = _paged_shapes(q, pool, page_table)
+    if tuple(scores.shape) != (B, T, N) or scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous fp32 [B][T][N]")
+    _check(lib().centroid_score_paged(ctx.handle, _ptr(q), _ptr(pool), nb, _ptr(page_table), N,
+                                      _ptr(lengths), B, T, Q, D, N, _ptr(scores),
+                                      _stream(stream, q.device)), "centroid_score_paged")
+    return scores
+
+
+def score_topk_fused_paged(ctx, q, pool, page_table, lengths, K, idx_out, val_out=None,
+                           stream=None):
+    """score_topk_fused with page p of request b read from pool[page_table[b, p]]."""
+    B, T, Q, D, N, nb = _paged_shapes(q, pool, page_table)
+    _check(lib().score_topk_fused_paged(ctx.handle, _ptr(q), _ptr(pool), nb, _ptr(page_table), N,
+                                        _ptr(lengths), B, T, Q, D, N, K, _ptr(idx_out),
+                                        _ptr(val_out), _stream(stream, q.device)),
+           "score_topk_fused_paged")
+    return idx_out, val_out

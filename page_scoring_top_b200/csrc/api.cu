@@ -102,10 +102,17 @@ int run_topk(idx_ctx* ctx, const float* scores, const int32_t* lengths, int len_
 // Scores into `scores` [B][T][N].  Per-token page counts (tok_lengths
 // [B*T], lengths unused) always take the decode kernels, which mask each
 // token row; the prefill kernel serves whole-request lengths only.
+// A paged table (page_table, non-null) also takes the decode kernels.
+struct Paged {
+  const int32_t* page_table = nullptr;
+  int64_t ld_pt = 0;
+  int n_blocks = 0;
+};
+
 int run_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t* lengths,
               const int32_t* tok_lengths, int B, int T, int Q, int D, int N, int64_t ldc_b,
-              float* scores, cudaStream_t stream) {
-  if (!tok_lengths && idx::prefill_supported(T, Q, D, ldc_b)) {
+              float* scores, cudaStream_t stream, const Paged& pg = Paged()) {
+  if (!tok_lengths && !pg.page_table && idx::prefill_supported(T, Q, D, ldc_b)) {
     for (int b0 = 0; b0 < B; b0 += idx::kPrefillMaxB) {
       idx::PrefillArgs p{};
       p.q = q + (int64_t)b0 * T * Q * D;
@@ -131,6 +138,12 @@ int run_score(idx_ctx* ctx, const uint16_t* q, const uint16_t* c, const int32_t*
     a.c = c + (int64_t)b0 * ldc_b;
     a.lengths = (lengths && !tok_lengths) ? lengths + b0 : nullptr;
     a.tok_lengths = tok_lengths ? tok_lengths + (int64_t)b0 * T : nullptr;
+    if (pg.page_table) {
+      a.c = c;  // the shared pool, not offset by request
+      a.page_table = pg.page_table + (int64_t)b0 * pg.ld_pt;
+      a.ld_pt = pg.ld_pt;
+      a.n_blocks = pg.n_blocks;
+    }
     a.B = nb;
     a.T = T;
     a.Q = Q;
@@ -273,7 +286,7 @@ IDX_API int topk_select(idx_ctx* ctx, const float* scores, const int32_t* length
 static int fused_impl(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
                       const int32_t* lengths, const int32_t* tok_lengths, int B, int T, int Q,
                       int D, int N, int64_t ldc_b, int K, int32_t* idx_out, float* val_out,
-                      idx_stream stream) {
+                      idx_stream stream, const Paged& pg = Paged()) {
   int rc = check_score_args(ctx, q, c, B, T, Q, D, N, ldc_b);
   if (rc != IDX_OK) return rc;
   if (!idx_out) return IDX_EINVAL;
@@ -283,7 +296,7 @@ static int fused_impl(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
   if (!guard.ok()) return IDX_ECUDA;
   cudaStream_t st = (cudaStream_t)stream;
   if (T <= idx::kDecodeMaxTFused && K <= idx::decode_fused_max_k(T) &&
-      (tok_lengths || !idx::prefill_supported(T, Q, D, ldc_b))) {
+      (tok_lengths || pg.page_table || !idx::prefill_supported(T, Q, D, ldc_b))) {
     for (int b0 = 0; b0 < B; b0 += idx::kDecodeMaxB) {
       const int nb = std::min(idx::kDecodeMaxB, B - b0);
       idx::DecodeArgs a{};
@@ -291,6 +304,12 @@ static int fused_impl(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
       a.c = c + (int64_t)b0 * ldc_b;
       a.lengths = (lengths && !tok_lengths) ? lengths + b0 : nullptr;
       a.tok_lengths = tok_lengths ? tok_lengths + (int64_t)b0 * T : nullptr;
+      if (pg.page_table) {
+        a.c = c;  // the shared pool, not offset by request
+        a.page_table = pg.page_table + (int64_t)b0 * pg.ld_pt;
+        a.ld_pt = pg.ld_pt;
+        a.n_blocks = pg.n_blocks;
+      }
       a.B = nb;
       a.T = T;
       a.Q = Q;
@@ -316,7 +335,7 @@ static int fused_impl(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
   // Prefill chunks (and token counts beyond the fused CUDA-core path): score
   // into the context's scratch, then select each (request, token) row.
   if ((int64_t)B * T * N > ctx->scratch_elems) return IDX_ENOWORKSPACE;
-  rc = run_score(ctx, q, c, lengths, tok_lengths, B, T, Q, D, N, ldc_b, ctx->scratch, st);
+  rc = run_score(ctx, q, c, lengths, tok_lengths, B, T, Q, D, N, ldc_b, ctx->scratch, st, pg);
   if (rc != IDX_OK) return rc;
   if (tok_lengths)  // one length per row
     return run_topk(ctx, ctx->scratch, tok_lengths, 1, B * T, N, N, K, idx_out, val_out, st);
@@ -354,6 +373,51 @@ IDX_API int score_topk_fused(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
                              idx_stream stream) {
   return fused_impl(ctx, q, c, lengths, nullptr, B, T, Q, D, N, ldc_b, K, idx_out, val_out,
                     stream);
+}
+
+// Paged entry points: `pool` holds n_blocks centroid rows of D values; the
+// row stride check of check_score_args is applied to a request stride of
+// N*D (the pool has no per-request rows).
+static int check_paged(const idx_ctx* ctx, const uint16_t* pool, const int32_t* page_table,
+                       int64_t ld_pt, int n_blocks, int N, int D) {
+  if (!ctx || !pool || !page_table) return IDX_EINVAL;
+  if (n_blocks <= 0 || ld_pt < N || N <= 0 || D <= 0) return IDX_EINVAL;
+  if (!aligned16(pool)) return IDX_EINVAL;
+  if ((D % 8) != 0 || D > 256) return IDX_EUNSUPPORTED;
+  return IDX_OK;
+}
+
+IDX_API int centroid_score_paged(idx_ctx* ctx, const uint16_t* q, const uint16_t* pool,
+                                 int n_blocks, const int32_t* page_table, int64_t ld_pt,
+                                 const int32_t* lengths, int B, int T, int Q, int D, int N,
+                                 float* scores, idx_stream stream) {
+  int rc = check_paged(ctx, pool, page_table, ld_pt, n_blocks, N, D);
+  if (rc != IDX_OK) return rc;
+  rc = check_score_args(ctx, q, pool, B, T, Q, D, N, (int64_t)N * D);
+  if (rc != IDX_OK) return rc;
+  if (!scores || !aligned16(scores)) return IDX_EINVAL;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  Paged pg;
+  pg.page_table = page_table;
+  pg.ld_pt = ld_pt;
+  pg.n_blocks = n_blocks;
+  return run_score(ctx, q, pool, lengths, nullptr, B, T, Q, D, N, (int64_t)N * D, scores,
+                   (cudaStream_t)stream, pg);
+}
+
+IDX_API int score_topk_fused_paged(idx_ctx* ctx, const uint16_t* q, const uint16_t* pool,
+                                   int n_blocks, const int32_t* page_table, int64_t ld_pt,
+                                   const int32_t* lengths, int B, int T, int Q, int D, int N,
+                                   int K, int32_t* idx_out, float* val_out, idx_stream stream) {
+  const int rc = check_paged(ctx, pool, page_table, ld_pt, n_blocks, N, D);
+  if (rc != IDX_OK) return rc;
+  Paged pg;
+  pg.page_table = page_table;
+  pg.ld_pt = ld_pt;
+  pg.n_blocks = n_blocks;
+  return fused_impl(ctx, q, pool, lengths, nullptr, B, T, Q, D, N, (int64_t)N * D, K, idx_out,
+                    val_out, stream, pg);
 }
 
 IDX_API int score_topk_fused_tokens(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,

@@ -28,6 +28,7 @@ namespace idx {
 // Written into the context's device status word; read by idx_get_status.
 constexpr int kErrLengthClamped = 1;  // a length outside [0, N] was clamped
 constexpr int kErrWaitTimeout = 2;    // a bounded wait gave up (data incomplete)
+constexpr int kErrPageClamped = 4;   // a page-table entry outside the block pool was clamped
 
 constexpr uint32_t kKeyInvalid = 0u;
 constexpr uint32_t kNegInfBits = 0xFF800000u;

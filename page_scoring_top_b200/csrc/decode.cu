@@ -189,6 +189,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
             if (*s_abort) continue;
             const uint32_t bytes = (uint32_t)min(kStagePages, np - sp) * page_bytes;
             mbar_arrive_expect_tx(&full[slot], bytes);
+            if (a.page_table) {
+              // paged: one copy per page from the shared block pool, no L2
+              // hint (pool rows are shared across requests and stay hot)
+              const int32_t* pt = a.page_table + (int64_t)b * a.ld_pt + p0 + sp;
+              const int n = min(kStagePages, np - sp);
+              for (int i = 0; i < n; ++i) {
+                int blk = __ldg(pt + i);
+                if (blk < 0 || blk >= a.n_blocks) {
+                  atomicOr(a.status, kErrPageClamped);
+                  blk = blk < 0 ? 0 : a.n_blocks - 1;
+                }
+                bulk_g2s_nohint(ring + (size_t)slot * stage_bytes + (size_t)i * page_bytes,
+                                a.c + (int64_t)blk * D, page_bytes, &full[slot]);
+              }
+              continue;
+            }
 #ifdef IDX_NO_L2_HINT
             bulk_g2s_nohint(ring + (size_t)slot * stage_bytes, src + (int64_t)sp * D, bytes,
                             &full[slot]);
@@ -383,8 +399,10 @@ static cudaError_t launch_tt(const DecodeArgs& a, int grid, cudaStream_t stream)
 cudaError_t launch_decode(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream) {
   // Head dims 64 and 128 with up to 64 query rows take the tensor-core kernel
   // (decode_tc.cu), in both modes so that fused and score-mode scores stay
-  // bit-identical; the CUDA-core kernel takes every other shape.
-  if (decode_tc_supported(a.T, a.Q, a.D, a.ldc_b, a.c)) return launch_decode_tc(a, fused, num_sms, stream);
+  // bit-identical; the CUDA-core kernel takes every other shape and every
+  // paged table (its producer copies page by page).
+  if (!a.page_table && decode_tc_supported(a.T, a.Q, a.D, a.ldc_b, a.c))
+    return launch_decode_tc(a, fused, num_sms, stream);
   const int grid = decode_grid(num_sms);
   if (fused) {
     if (a.D == 128) return launch_tt<128, true>(a, grid, stream);

@@ -37,6 +37,11 @@ struct DecodeArgs {
   const uint16_t* c;
   const int32_t* lengths;      // per request, or null
   const int32_t* tok_lengths;  // per (request, token) [B*T] instead of lengths, or null
+  // paged centroids: page p of request b is row page_table[b*ld_pt + p] of
+  // the block pool `c` ([n_blocks][D]); null for contiguous per-request rows
+  const int32_t* page_table;
+  int64_t ld_pt;
+  int n_blocks;
   int B, T, Q, D, N;
   int64_t ldc_b;
   int K;

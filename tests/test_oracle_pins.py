@@ -435,3 +435,24 @@ def test_pool_closed_forms():
     # a library mean over the same keys
     lib = kf[1, 20:23].mean(axis=0)
     assert np.allclose(oracle.pool(k, counts, 4, 10)[1, 5], lib, rtol=0, atol=1e-15)
+
+
+# ------------------------------------------------------------------ paged centroid table
+
+def test_paged_scores_gather_the_pool():
+    # a pool of 3 blocks; request 0 reads blocks [2, 0, 2], request 1 reads [1]
+    q = _bf16([[[[1.0, 2.0]]], [[[0.5, -1.0]]]])          # [2][1][1][2]
+    pool = _bf16([[1.0, 0.0], [0.0, 1.0], [3.0, 1.0]])     # [3][2]
+    pt = np.array([[2, 0, 2], [1, 0, 0]], np.int32)
+    S, _ = oracle.scores_paged(q, pool, pt, np.array([3, 1], np.int32))
+    assert S[0, 0].tolist() == [5.0, 1.0, 5.0]
+    assert S[1, 0].tolist() == [-1.0, -np.inf, -np.inf]
+
+
+def test_paged_identity_table_equals_contiguous():
+    d = synth.decode_inputs(41, B=2, T=1, Q=2, D=16, N=30, lengths=[30, 17])
+    pool = d["c"].reshape(60, 16)
+    pt = np.arange(60, dtype=np.int32).reshape(2, 30)
+    S1, A1 = oracle.scores(d["q"], d["c"], d["lengths"])
+    S2, A2 = oracle.scores_paged(d["q"], pool, pt, d["lengths"])
+    assert np.array_equal(S1, S2) and np.array_equal(A1, A2)
