@@ -169,6 +169,45 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   // k % kProducerLanes): one issuing thread alone caps the copy rate well
   // below HBM bandwidth.  The ring depth is a multiple of kProducerLanes, so a
   // slot is always refilled by the same lane, in order.
+  if (warp == kConsumerWarps && a.page_table) {
+    // Paged table: the whole warp fills each stage, lane i copying page i of
+    // the stage from its block-pool row (no L2 hint: pool rows are shared
+    // across requests and stay hot).  Entries outside the pool are clamped.
+    uint32_t stage = 0;
+    for (int j = g; j < nchunks; j += G) {
+      const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
+      const int b_last = ch.row(ce - 1);
+      for (int b = ch.row(cb); b <= b_last; ++b) {
+        if (ch.len(b) == 0) continue;
+        const int p0 = ch.snap(b, cb);
+        const int np = ch.snap(b, ce) - p0;
+        const int32_t* pt = a.page_table + (int64_t)b * a.ld_pt + p0;
+        for (int sp = 0; sp < np; sp += kStagePages, ++stage) {
+          const int slot = (int)(stage % (uint32_t)nst);
+          const uint32_t round = stage / (uint32_t)nst;
+          int go = 1;
+          if (lane == 0) {
+            if (round > 0) mbar_wait_bounded(&empty[slot], (round - 1) & 1, s_abort, a.status);
+            go = *s_abort == 0;
+          }
+          go = __shfl_sync(0xFFFFFFFFu, go, 0);
+          if (!go) continue;
+          const int n = min(kStagePages, np - sp);
+          if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)n * page_bytes);
+          if (lane < n) {
+            int blk = __ldg(pt + sp + lane);
+            if (blk < 0 || blk >= a.n_blocks) {
+              atomicOr(a.status, kErrPageClamped);
+              blk = blk < 0 ? 0 : a.n_blocks - 1;
+            }
+            bulk_g2s_nohint(ring + (size_t)slot * stage_bytes + (size_t)lane * page_bytes,
+                            a.c + (int64_t)blk * D, page_bytes, &full[slot]);
+          }
+        }
+      }
+    }
+    return;
+  }
   if (warp == kConsumerWarps) {
     if (lane < kProducerLanes) {
       const uint64_t pol = policy_evict_first();
@@ -189,22 +228,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
             if (*s_abort) continue;
             const uint32_t bytes = (uint32_t)min(kStagePages, np - sp) * page_bytes;
             mbar_arrive_expect_tx(&full[slot], bytes);
-            if (a.page_table) {
-              // paged: one copy per page from the shared block pool, no L2
-              // hint (pool rows are shared across requests and stay hot)
-              const int32_t* pt = a.page_table + (int64_t)b * a.ld_pt + p0 + sp;
-              const int n = min(kStagePages, np - sp);
-              for (int i = 0; i < n; ++i) {
-                int blk = __ldg(pt + i);
-                if (blk < 0 || blk >= a.n_blocks) {
-                  atomicOr(a.status, kErrPageClamped);
-                  blk = blk < 0 ? 0 : a.n_blocks - 1;
-                }
-                bulk_g2s_nohint(ring + (size_t)slot * stage_bytes + (size_t)i * page_bytes,
-                                a.c + (int64_t)blk * D, page_bytes, &full[slot]);
-              }
-              continue;
-            }
 #ifdef IDX_NO_L2_HINT
             bulk_g2s_nohint(ring + (size_t)slot * stage_bytes, src + (int64_t)sp * D, bytes,
                             &full[slot]);
