@@ -57,13 +57,12 @@ def _load():
         lib.oracle_scores.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
         lib.oracle_scores_tokens.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
         lib.oracle_pool.argtypes = [P, P, I, I, I, I, L, P]
-        lib.oracle_scores_at.argtypes = [P, P, I, I, I, I, I, L, L, P, P, P, P, P]
         lib.oracle_topk_f64.argtypes = [P, I, I, P, P]
         lib.oracle_topk_f32.argtypes = [P, I, I, P, P]
         lib.oracle_topk_rows_f32.argtypes = [P, P, I, I, L, I, P, P]
         lib.oracle_topk_rows_f64.argtypes = [P, P, I, I, L, I, P, P]
-        for f in ("oracle_scores", "oracle_scores_tokens", "oracle_pool", "oracle_scores_at", "oracle_topk_f64", "oracle_topk_f32",
-                  "oracle_topk_rows_f32", "oracle_topk_rows_f64"):
+        for f in ("oracle_scores", "oracle_scores_tokens", "oracle_pool", "oracle_topk_f64",
+                  "oracle_topk_f32", "oracle_topk_rows_f32", "oracle_topk_rows_f64"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -127,30 +126,16 @@ def scores_paged(q_bits, pool_bits, page_table, lengths=None):
     pool = _c(pool_bits, np.uint16)
     pt = np.asarray(page_table)
     B, N = pt.shape
-    gathered = pool[np.clip(pt, 0, pool.shape[0] - 1)]  # [B][N][D]
+    live = np.ones((B, N), bool)
     if lengths is not None:
         live = np.arange(N)[None, :] < np.asarray(lengths)[:, None]
-        gathered = np.where(live[:, :, None], gathered, np.uint16(0))
+    # The page only defines a table of valid block ids: an id outside the pool
+    # on a live page has no meaning, so it is an error here, not a value.
+    if np.any(live & ((pt < 0) | (pt >= pool.shape[0]))):
+        raise ValueError("scores_paged: page-table entry outside the block pool")
+    gathered = pool[np.where(live, pt, 0)]  # [B][N][D]; dead pages read block 0, then masked
+    gathered = np.where(live[:, :, None], gathered, np.uint16(0))
     return scores(q_bits, gathered, lengths)
-
-
-def scores_at(q_bits, c_bits, b, t, p):
-    """Exact S and A at the listed (b, t, p) triples (spot checks at full size)."""
-    q = _c(q_bits, np.uint16)
-    c = _c(c_bits, np.uint16)
-    B, T, Q, D = q.shape
-    _, N, _ = c.shape
-    b = _c(b, np.int32)
-    t = _c(t, np.int32)
-    p = _c(p, np.int32)
-    n = b.size
-    S = np.empty(n, np.float64)
-    A = np.empty(n, np.float64)
-    rc = _load().oracle_scores_at(_ptr(q), _ptr(c), B, T, Q, D, N, N * D, n,
-                                  _ptr(b), _ptr(t), _ptr(p), _ptr(S), _ptr(A))
-    if rc != 0:
-        raise ValueError("oracle_scores_at: arguments outside the contract")
-    return S, A
 
 
 def topk(row, K, length=None):

@@ -142,24 +142,6 @@ ORACLE_API int oracle_scores_tokens(const uint16_t* q, const uint16_t* c,
     return 0;
 }
 
-/* Scores at n listed (b, t, p) triples, for spot checks at full size. */
-ORACLE_API int oracle_scores_at(const uint16_t* q, const uint16_t* c, int B,
-                                int T, int Q, int D, int N, int64_t ldc_b,
-                                int64_t n, const int32_t* bb, const int32_t* tt,
-                                const int32_t* pp, double* S, double* A)
-{
-    if (Q <= 0 || D <= 0 || n < 0) return -1;
-    for (int64_t i = 0; i < n; ++i) {
-        if (bb[i] < 0 || bb[i] >= B || tt[i] < 0 || tt[i] >= T || pp[i] < 0 ||
-            pp[i] >= N)
-            return -1;
-        score_one(q + ((int64_t)bb[i] * T + tt[i]) * Q * D,
-                  c + (int64_t)bb[i] * ldc_b + (int64_t)pp[i] * D, Q, D, &S[i],
-                  &A[i]);
-    }
-    return 0;
-}
-
 typedef struct {
     double v;
     int32_t i;

@@ -456,3 +456,17 @@ def test_paged_identity_table_equals_contiguous():
     S1, A1 = oracle.scores(d["q"], d["c"], d["lengths"])
     S2, A2 = oracle.scores_paged(d["q"], pool, pt, d["lengths"])
     assert np.array_equal(S1, S2) and np.array_equal(A1, A2)
+
+
+def test_paged_scores_reject_ids_outside_the_pool():
+    # The block-pool table ("Iterate Centroids Score", the ctx argument)
+    # names valid blocks only: a live page pointing outside the pool is an
+    # error for the oracle, while entries past a request's length are never read.
+    q = _bf16([[[[1.0, 2.0]]]])
+    pool = _bf16([[1.0, 0.0], [0.0, 1.0]])
+    with pytest.raises(ValueError):
+        oracle.scores_paged(q, pool, np.array([[0, 2]], np.int32), np.array([2], np.int32))
+    with pytest.raises(ValueError):
+        oracle.scores_paged(q, pool, np.array([[-1, 0]], np.int32), np.array([2], np.int32))
+    S, _ = oracle.scores_paged(q, pool, np.array([[1, 99]], np.int32), np.array([1], np.int32))
+    assert S[0, 0].tolist() == [2.0, -np.inf]
