@@ -48,11 +48,11 @@ NOMINAL_HBM_GBS = 8000.0
 KERNEL = "decode_tc_kernel<D=128,NC=16,fused,hist>"
 PREFILL_KERNEL = "prefill_kernel<Q=8> (tcgen05 score of a 16-token chunk)"
 FALLBACK_HBM_GBS = 6650.0
-# DRAM bytes per valid page of the fused decode kernel, from the ncu capture
-# summarised in profiles/decode_fused_ragged_decode.md: (301.27 MB read +
-# 3.47 MB written) per launch / 1,175,731 pages.  Set to None whenever the
-# kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES_PER_PAGE = 259.2
+# The ncu summary of the headline kernel records its DRAM bytes per valid page
+# beside a digest of the library sources it was captured on; the traffic is
+# reported only while the sources still have that digest.
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "decode_fused_ragged_decode.md")
+REPEATS = 11  # timed regions of exactly --steps steps; the median is reported
 
 
 def parse():
@@ -67,8 +67,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=("ragged_decode", "prefill_chunk", "causal_decode", "pool_keys",
-                             "paged_decode",
+                             "paged_decode", "topk_sweep",
                              "batch_decode_bias", "tiny_decode"))
+    ap.add_argument("--dists", default="normal,levels16,neg_inf_90",
+                    help="top-K sweep distributions (comma list, or 'all')")
     return ap.parse_args()
 
 
@@ -93,6 +95,79 @@ def algorithmic_bytes(lengths, B, T, Q, D, K, with_values):
     if with_values:
         b += B * T * K * 4
     return pages, b
+
+
+def source_digest():
+    """sha256 (first 16 hex digits) over the library's CUDA sources and header."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "page_scoring_top_b200", "csrc", "*")))
+    for f in files + [os.path.join(ROOT, "include", "idx.h")]:
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic_per_page():
+    """(bytes per valid page, note) from the committed ncu summary, or (None,
+    why) when the summary is missing or the sources changed since its capture."""
+    import re
+    try:
+        with open(TRAFFIC_SUMMARY) as f:
+            text = f.read()
+    except OSError:
+        return None, "no ncu summary"
+    m = re.search(r"traffic_bytes_per_page\s*=\s*([0-9.]+)\s*;\s*sources\s*=\s*([0-9a-f]+)", text)
+    if not m:
+        return None, "no traffic record in the ncu summary"
+    if m.group(2) != source_digest():
+        return None, "kernel sources changed since the ncu capture"
+    return float(m.group(1)), "ncu capture of this kernel build (dram read + write per page)"
+
+
+def host_facts():
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+def timed_repeats(step, steps, stream, barrier, repeats=REPEATS):
+    """``repeats`` timed regions of exactly ``steps`` steps, each bracketed by
+    a barrier and a device synchronize on both sides and timed with CUDA
+    events on the launching stream.  Returns the per-region milliseconds."""
+    import torch
+    out = []
+    for _ in range(repeats):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        out.append(e0.elapsed_time(e1))
+    return out
+
+
+def soak(step, seconds):
+    """Run untimed steps for about ``seconds`` (the clock sampler's window)."""
+    import torch
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        for _ in range(50):
+            step()
+        torch.cuda.synchronize()
 
 
 def measured_peak():
@@ -223,7 +298,7 @@ def run_reference(args):
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": "per step: the first %d valid pages of one request "
                                    "(requests in turn), scores in double + full sort" %
-                                   sample_pages},
+                                   sample_pages, **host_facts()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -282,26 +357,29 @@ def run_ours(args):
         if pg is not None:
             pg.barrier()
 
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else
                            os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
     barrier()
     torch.cuda.synchronize(dev)
+    # The sampler covers a window of load around the timed regions, so that
+    # the clock record holds more than one reading even for short regions.
     sampler.start()
     time.sleep(0.15)  # let the sampler take its first reading
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
+    soak(step, 0.3)
+    reps = timed_repeats(step, args.steps, stream, barrier)
+    soak(step, 0.3)
     clocks = sampler.stop()
-    barrier()
-    ms = ev0.elapsed_time(ev1)
     from page_scoring_top_b200 import dist as pdist
-    ms_max, total_pages = pdist.reduce_timing(ms, units, device=dev)
+    reps_max = [pdist.reduce_timing(r, units, device=dev)[0] for r in reps]
+    ms_max = float(np.median(reps_max))
+    total_pages = pdist.reduce_timing(0.0, units, device=dev)[1]
+    ms = float(np.median(reps))  # this rank's own median region
     ms_per_step = ms_max / args.steps
     value = total_pages * args.steps / (ms_max * 1e-3)
+    repeats = {"regions": len(reps_max), "steps_each": args.steps,
+               "ms_per_step": [r / args.steps for r in reps_max],
+               "median_ms_per_step": ms_per_step,
+               "spread": (max(reps_max) - min(reps_max)) / ms_max}
     rc, bits = binding.idx_get_status(ctx)
     if rc != 0:
         raise RuntimeError("device status %d after the timed region" % bits)
@@ -311,9 +389,10 @@ def run_ours(args):
     # the step is the tcgen05 score kernel then the top-K kernel; the score
     # kernel (centroid_score alone) is timed the same way on the same stream.
     peak, peak_src = measured_peak()
-    kernel, traffic = KERNEL, None
-    if args.workload == WORKLOAD and NCU_TRAFFIC_BYTES_PER_PAGE is not None:
-        traffic = NCU_TRAFFIC_BYTES_PER_PAGE * pages
+    kernel, traffic, traffic_note = KERNEL, None, "no ncu capture for this workload"
+    if args.workload == WORKLOAD:
+        per_page, traffic_note = recorded_traffic_per_page()
+        traffic = None if per_page is None else per_page * pages
     launch_s = (ms / args.steps) * 1e-3
     score_bytes = nbytes
     tensor = None
@@ -346,7 +425,8 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         rate, sample = cpu_oracle_rate(d, K, args.cpu_seconds)
-        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
+        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+               **host_facts()}
 
     if rank == 0:
         line = {
@@ -365,9 +445,10 @@ def run_ours(args):
                              "no flush" % (pages * D * 2 / 1e6)},
             "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "kernel": kernel},
+                         "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_note,
+                         "peak_source": peak_src, "kernel": kernel},
             "gpu_launches": args.steps * (2 if (T > 1 and tok is None) else 1),
+            "repeats": repeats,
             "clocks": clocks,
             "tensor": tensor,
             "e2e": e2e,
@@ -553,6 +634,85 @@ def run_paged(args):
     return 0
 
 
+def run_topk_sweep(args):
+    """The standalone top-K sweep: fp32 score rows, rows in {1, 8, 32, 128} x
+    N in {4096, 16384, 65536, 262144}, K = 256, each case with its own seed
+    (104 + case number).  One topk_select call per step.  Cases whose rows
+    fit in L2 get a 256 MB L2 flush before every timed call (each call timed
+    alone with CUDA events); larger ones run back to back.  Prints one line
+    with every case's time and HBM fraction (rows * (N + K) * 4 bytes)."""
+    import torch
+    from page_scoring_top_b200 import binding, synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    K = 256
+    dists = synth.DISTRIBUTIONS if args.dists == "all" else tuple(args.dists.split(","))
+    peak, peak_src = measured_peak()
+    ctx = binding.Context(0, max_rows=max(synth.SWEEP_ROWS), max_n=max(synth.SWEEP_N), max_k=K)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    l2_bytes = 126 << 20
+    steps = max(3, min(args.steps, 200))
+    cases = []
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.15)
+    for case, rows, n, dist in synth.sweep_cases():
+        if dist not in dists:
+            continue
+        s = torch.from_numpy(synth.score_rows(104 + case, rows, n, dist)).to(dev)
+        idx = torch.empty((rows, K), dtype=torch.int32, device=dev)
+        call = lambda: binding.topk_select(ctx, s, None, K, idx, None, stream=stream)
+        for _ in range(max(3, args.warmup)):
+            call()
+        nbytes = rows * (n + K) * 4
+        per = []
+        if nbytes < l2_bytes:
+            for _ in range(steps):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                call()
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                per.append(e0.elapsed_time(e1))
+            ms = float(np.median(per))
+        else:
+            ms = float(np.median(timed_repeats(call, steps, stream, lambda: None, 5))) / steps
+        rc, bits = binding.idx_get_status(ctx)
+        if rc != 0:
+            raise RuntimeError("device status %d" % bits)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        cases.append({"case": case, "rows": rows, "N": n, "dist": dist, "us": ms * 1e3,
+                      "rows_per_s": rows / (ms * 1e-3), "hbm_gbs": gbs, "frac": gbs / peak,
+                      "l2": "flushed" if nbytes < l2_bytes else "larger than L2"})
+        del s, idx
+    clocks = sampler.stop()
+    big = [c for c in cases if c["rows"] * c["N"] * 4 >= (32 << 20)]
+    head = max(cases, key=lambda c: (c["rows"] * c["N"], c["frac"]))
+    line = {
+        "metric": "top-K rows selected/sec (standalone select, fp32 rows, K=256)",
+        "value": head["rows_per_s"], "unit": "rows/s", "n_gpus": 1, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": head["us"] * 1e-3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "topk_sweep", "K": K, "dists": list(dists),
+                   "value_case": "rows=%d N=%d %s" % (head["rows"], head["N"], head["dist"]),
+                   "l2": "flush (256 MB write) before each call below 126 MB; larger cases "
+                         "back to back"},
+        "roofline": {"bound": "hbm", "achieved": head["hbm_gbs"], "peak": peak, "unit": "GB/s",
+                     "frac": head["frac"], "traffic": None, "peak_source": peak_src,
+                     "kernel": "topk select (standalone)",
+                     "median_frac_cases_ge_32MB": float(np.median([c["frac"] for c in big]))
+                     if big else None},
+        "gpu_launches": None, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+        "cases": cases,
+    }
+    print(json.dumps(line), flush=True)
+    ctx.close()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -561,6 +721,8 @@ def main():
         return run_pool(args)
     if args.workload == "paged_decode":
         return run_paged(args)
+    if args.workload == "topk_sweep":
+        return run_topk_sweep(args)
     return run_ours(args)
 
 

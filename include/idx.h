@@ -195,12 +195,14 @@ IDX_API int idx_num_sms(const idx_ctx* ctx);
 
 /*
  * topk_select without a context, for callers that cannot allocate device
- * memory: code running while a CUDA graph is captured, serving engines that
- * plan all device memory up front, plugin hosts that provide no allocator.
+ * memory: serving engines that plan all device memory up front and forbid
+ * allocation on the request path, and plugin hosts that hand a library
+ * device pointers but no allocator.
  * The pages have no counterpart of this call; it exists for those callers.
  *
- * Same arguments, result and error codes as topk_select, on the calling
- * thread's current device.  Its scratch (candidate lists, per-row counters)
+ * Same arguments and result as topk_select, on the calling thread's current
+ * device, and the same error codes except IDX_EDEVICE, which this call never
+ * returns: it has no status word to read.  Its scratch (candidate lists, per-row counters)
  * is one static 8 MiB device array that every GPU loading the library holds
  * until the process exits; rows x ceil(N / chunk) x K candidate entries must
  * fit in it (about 1M entries), else IDX_ENOWORKSPACE.  The call allocates
@@ -208,7 +210,9 @@ IDX_API int idx_num_sms(const idx_ctx* ctx);
  * (do that first call before any stream capture), and every call clears the
  * counters it uses with cudaMemsetAsync on `stream`.  All calls share the
  * array, which keeps the last call's contents, so calls that overlap on the
- * GPU race; clamped lengths are not reported (there is no status to read).
+ * GPU race.  Lengths outside [0, N] are clamped as in topk_select but not
+ * reported.  The first-call set-up is safe when several host threads make
+ * their first calls at once.
  */
 IDX_API int topk_select_noalloc(const float* scores, const int32_t* lengths, int rows, int N,
                                 int64_t lds, int K, int32_t* idx_out, float* val_out,

@@ -171,9 +171,12 @@ def topk_select_noalloc(scores, lengths, K, idx_out, val_out=None, stream=None):
     if scores.dim() != 2 or scores.stride(1) != 1:
         raise ValueError("scores must be 2-D with unit column stride")
     rows, N = scores.shape
-    _check(lib().topk_select_noalloc(_ptr(scores), _ptr(lengths), rows, N, scores.stride(0), K,
-                                     _ptr(idx_out), _ptr(val_out), _stream(stream, scores.device)),
-           "topk_select_noalloc")
+    # the C call works on the current device: make it the one holding the data
+    with torch.cuda.device(scores.device):
+        _check(lib().topk_select_noalloc(_ptr(scores), _ptr(lengths), rows, N, scores.stride(0),
+                                         K, _ptr(idx_out), _ptr(val_out),
+                                         _stream(stream, scores.device)),
+               "topk_select_noalloc")
     return idx_out, val_out
 
 

@@ -35,19 +35,30 @@ def stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compile every csrc/*.cu to an object (in parallel), then link libidx.so."""
     if not force and not stale():
         return LIB
+    import concurrent.futures
+    import tempfile
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [nvcc, "-O3", "-std=c++17", *ARCH, "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
-           "-I", os.path.join(ROOT, "include"), *extra, *sources(), "-o", tmp]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    flags = ["-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
+             "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
+             "-I", os.path.join(ROOT, "include"), *extra]
+    with tempfile.TemporaryDirectory(prefix="idx_build_") as tmpdir:
+        def compile_one(src):
+            obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+            cmd = [nvcc, *flags, "-c", src, "-o", obj]
+            if verbose:
+                print(" ".join(cmd), file=sys.stderr)
+            subprocess.check_call(cmd)
+            return obj
+        srcs = sources()
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
+            objs = list(ex.map(compile_one, srcs))
+        tmp = LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call([nvcc, "-shared", *ARCH, *objs, "-o", tmp])
+        os.replace(tmp, LIB)
     return LIB
-
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,

@@ -119,6 +119,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Bounded wait that ignores the abort flag: a producer draining its own copies
+// in flight before the CTA exits.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kMaxWaitIters; ++it)
+    if (mbar_try_wait(bar, parity)) return;
+}
+
 // Programmatic dependent launch.  launch_dependents lets the next kernel of
 // the stream, when it was launched as a programmatic dependent, start
 // launching (its CTAs take SMs as this grid's CTAs exit); wait blocks until

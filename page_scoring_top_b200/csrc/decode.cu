@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
     // the stage from its block-pool row (no L2 hint: pool rows are shared
     // across requests and stay hot).  Entries outside the pool are clamped.
     uint32_t stage = 0;
+    int64_t last = -1;  // last stage this warp filled
     for (int j = g; j < nchunks; j += G) {
       const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
       const int b_last = ch.row(ce - 1);
@@ -203,15 +204,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
             bulk_g2s_nohint(ring + (size_t)slot * stage_bytes + (size_t)lane * page_bytes,
                             a.c + (int64_t)blk * D, page_bytes, &full[slot]);
           }
+          last = stage;
         }
       }
     }
+    // Nothing may still be landing in shared memory when the CTA exits (this
+    // matters only after an abort): wait for the last stages' copies.
+    if (lane == 0)
+      for (int64_t t = last; t >= 0 && t > last - nst; --t)
+        mbar_wait_drain(&full[t % nst], (uint32_t)(t / nst) & 1);
     return;
   }
   if (warp == kConsumerWarps) {
     if (lane < kProducerLanes) {
       const uint64_t pol = policy_evict_first();
       uint32_t stage = 0;
+      int64_t last = -1;  // last stage this lane issued
       for (int j = g; j < nchunks; j += G) {
         const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
         const int b_last = ch.row(ce - 1);
@@ -236,9 +244,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
             bulk_g2s(ring + (size_t)slot * stage_bytes, src + (int64_t)sp * D, bytes, &full[slot],
                      pol);
 #endif
+            last = stage;
           }
         }
       }
+      // As above: wait for this lane's copies still in flight before exiting.
+      for (int64_t t = last; t >= 0 && t > last - nst; t -= kProducerLanes)
+        mbar_wait_drain(&full[t % nst], (uint32_t)(t / nst) & 1);
     }
     return;
   }

@@ -109,12 +109,6 @@ __host__ __device__ inline TcLayout tc_layout(bool fused, int D, int T, int Q) {
   return L;
 }
 
-// Bounded wait that ignores the abort flag (draining copies in flight).
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kMaxWaitIters; ++it)
-    if (mbar_try_wait(bar, parity)) return;
-}
-
 // D: head dim (64 or 128).  NC: query rows the epilogue unrolls (16 or 64).
 // HIST: single-token fused rows with the histogram select.
 template <int D, int NC, bool FUSED, bool HIST>
@@ -297,6 +291,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int wg = warp >> 2;    // warpgroup: takes tiles with (tile & 1) == wg
     const int quad = warp & 3;   // TMEM lanes quad*32 .. quad*32+31 = pages of the tile
+    IDX_TRACE(10);
     if (!FUSED) score_padding(a, s_off, g, G);
     else fused_empty_rows(a, s_off, g, G);
     const int rows = T * Q;
@@ -396,6 +391,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             next_check = tt + max(1, fused_check<HIST>(fsel, T, a.K, compact_at) / kTcTile);
           }
         }
+        IDX_TRACE(12);
         if (FUSED) fused_finalize<HIST>(fsel, a, T, b, j, ch.first(b), ch.last(b));
       }
     }

@@ -127,6 +127,7 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
     float* out_v = a.val_out ? a.val_out + (int64_t)b * a.K : nullptr;
     const int64_t slot = (int64_t)(j + b);
     hist_scan<kSelThreads>(f.hist, start, (uint32_t)a.K, sc);
+    IDX_TRACE(13);
     if (sc.bcast[0] == 0xFFFFFFFFu || sc.bcast[2] <= (uint32_t)kBoundaryMax) {
       constexpr int E = kFilterCap / kSelThreads;
       uint64_t v[E];
@@ -150,7 +151,9 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
                                         a.cand_bits + slot * a.slot_stride,
                                         a.cand_idx + slot * a.slot_stride, a.row_thr + b);
     }
+    IDX_TRACE(14);
     if (!single && arrive_last<kSelThreads>(a.arrive + b, j1 - j0 + 1, f.s_flag)) {
+      IDX_TRACE(15);
       const int nslots = j1 - j0 + 1;
       auto slot_of = [=](int i) { return (int64_t)(j0 + i + b); };
       bool done = false;
@@ -162,6 +165,7 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
         merge_candidates<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride,
                                       a.K, a.row_thr + b, fs, f.fbuf, f.fbuf + kFilterCap,
                                       kFilterCap, sc, f.sortv, f.sortb, out_i, out_v);
+      IDX_TRACE(16);
     }
   } else {
     for (int t = 0; t < T; ++t) {

@@ -1,10 +1,8 @@
 // noalloc.cu -- topk_select for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc: code that runs while a CUDA graph is
-// being captured (an allocation there breaks or invalidates the capture),
-// serving engines that plan every byte of device memory up front and forbid
-// allocations on the request path, and plugin hosts that hand a library
-// device pointers but no allocator.  topk_select needs scratch for the
+// Some callers cannot call cudaMalloc: serving engines that plan every byte
+// of device memory up front and forbid allocations on the request path, and
+// plugin hosts that hand a library device pointers but no allocator.  topk_select needs scratch for the
 // per-chunk candidate lists of long rows and for the per-row counters; this
 // variant keeps that scratch in one file-scope static device array instead of
 // an idx_ctx workspace, so the call itself allocates nothing.
@@ -16,7 +14,9 @@
 // calls share the array and it keeps the last call's contents: each call
 // clears the counters it needs (cudaMemsetAsync on the caller's stream), and
 // calls that overlap on the GPU (other streams, other host threads) race.
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "idx.h"
@@ -29,8 +29,32 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-unsigned char* g_scratch_addr[kMaxDevices] = {};
+// Per-device set-up results.  Host threads may make their first calls at the
+// same time: the set-up runs under a mutex, and the address is published with
+// release order after the SM count, so a thread that reads a non-null address
+// (acquire) also sees that device's SM count.
+std::atomic<unsigned char*> g_scratch_addr[kMaxDevices] = {};
 int g_scratch_sms[kMaxDevices] = {};
+std::mutex g_setup_mutex;
+
+// The device address of the scratch array on the current device `dev`
+// (looked up once per device), or null on a CUDA error.
+unsigned char* scratch_on(int dev) {
+  unsigned char* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  p = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return nullptr;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return nullptr;
+  g_scratch_sms[dev] = sms;
+  p = static_cast<unsigned char*>(addr);
+  g_scratch_addr[dev].store(p, std::memory_order_release);
+  return p;
+}
 
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -45,16 +69,8 @@ extern "C" IDX_API int topk_select_noalloc(const float* scores, const int32_t* l
   if (K > IDX_MAX_K) return IDX_EUNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return IDX_ECUDA;
-  if (!g_scratch_addr[dev]) {  // set-up, once per device, with that device current
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return IDX_ECUDA;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return IDX_ECUDA;
-    g_scratch_sms[dev] = sms;
-    g_scratch_addr[dev] = static_cast<unsigned char*>(p);
-  }
-  unsigned char* base = g_scratch_addr[dev];
+  unsigned char* base = scratch_on(dev);  // set-up, once per device, with that device current
+  if (!base) return IDX_ECUDA;
   idx::TopkArgs a{};
   a.chunk = idx::topk_plan_chunk(rows, N, K, g_scratch_sms[dev]);
   a.max_chunks = (N + a.chunk - 1) / a.chunk;

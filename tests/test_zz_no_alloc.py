@@ -1,6 +1,6 @@
 """topk_select_noalloc: the context-free variant for callers that cannot
-allocate device memory (graph capture, engines that plan all memory up front,
-plugin hosts without an allocator).  Its scratch is a static device array, so
+allocate device memory (engines that plan all memory up front, plugin hosts
+without an allocator).  Its scratch is a static device array, so
 this test checks, through the C ABI, that two calls in a row -- the second on
 a different shape, after the first left its contents in the shared array --
 give exactly what topk_select gives."""
@@ -39,6 +39,16 @@ def test_noalloc_matches_topk_select_on_two_calls():
         torch.cuda.synchronize()
         assert torch.equal(got_i, ref_i)
         assert torch.equal(got_v.view(torch.int32), ref_v.view(torch.int32))
+    # the Python wrapper runs the same call on the tensor's device
+    s, K = synth.score_rows(4244, 3, 5000, "uniform"), 64
+    sd = to_dev(s)
+    ref_i, ref_v = poisoned_outputs(3, K)
+    binding.topk_select(ctx, sd, None, K, ref_i, ref_v)
+    got_i, got_v = poisoned_outputs(3, K)
+    binding.topk_select_noalloc(sd, None, K, got_i, got_v)
+    torch.cuda.synchronize()
+    assert torch.equal(got_i, ref_i)
+    assert torch.equal(got_v.view(torch.int32), ref_v.view(torch.int32))
     # beyond the scratch limit: a clear error, nothing launched
     # (256 rows x 4 chunks x K = 2048 candidates: 2M entries, twice the limit)
     big = torch.zeros((256, 65536), device="cuda")
