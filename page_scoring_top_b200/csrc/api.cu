@@ -19,10 +19,13 @@ struct idx_ctx {
   int num_sms;
   void* ws;  // one allocation holding everything below
   size_t ws_bytes;
-  uint32_t* cand_bits;
+  uint32_t* cand_bits;  // standalone select: cand_slots lists of max_k entries
   int32_t* cand_idx;
-  unsigned long long* row_thr;
   int64_t cand_slots;
+  uint32_t* fcand_bits;  // fused decode: fused_slots lists of fused_stride entries
+  int32_t* fcand_idx;
+  int64_t fused_slots, fused_stride;
+  unsigned long long* row_thr;
   int32_t* arrive;
   int* status;
   float* scratch;  // fp32 scores for the score-then-select route
@@ -181,9 +184,11 @@ IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max
   ctx->max_n = max_n;
   ctx->max_k = max_k;
   ctx->num_sms = sms;
-  // Candidate slots: the larger of the standalone select's (rows x chunks of
-  // at least 2048 entries) and the fused decode path's (chunks + requests).
-  const int64_t topk_slots = (int64_t)max_rows * ceil_div(max_n, 2048);
+  // Candidate slots of the standalone select: rows x chunks of at least 2048
+  // entries, K entries each.  The fused decode path has its own slots (chunks
+  // + requests), wider: a segment publishes about K entries plus one digit
+  // bin's worth.
+  ctx->cand_slots = (int64_t)max_rows * ceil_div(max_n, 2048);
   int64_t fused_slots = 0;
   for (int t = 1; t <= idx::kDecodeMaxTFused; ++t) {
     const int64_t b = std::min<int64_t>(max_rows / t, idx::kDecodeMaxB);
@@ -191,7 +196,9 @@ IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max
       fused_slots = std::max(fused_slots,
                              idx::decode_fused_slots(b, t, max_n, idx::decode_grid(sms)));
   }
-  ctx->cand_slots = std::max(topk_slots, fused_slots);
+  ctx->fused_slots = fused_slots;
+  // (a multiple of 4 entries: lists are copied 16 bytes at a time)
+  ctx->fused_stride = ((int64_t)max_k + std::max(max_k, 256) + 3) & ~(int64_t)3;
   ctx->scratch_elems = (int64_t)max_rows * max_n;
   size_t off = 0;
   auto carve = [&](size_t bytes) {
@@ -201,6 +208,8 @@ IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max
   };
   const size_t o_bits = carve((size_t)ctx->cand_slots * max_k * 4);
   const size_t o_idx = carve((size_t)ctx->cand_slots * max_k * 4);
+  const size_t o_fbits = carve((size_t)ctx->fused_slots * ctx->fused_stride * 4);
+  const size_t o_fidx = carve((size_t)ctx->fused_slots * ctx->fused_stride * 4);
   const size_t o_thr = carve((size_t)max_rows * 8);
   const size_t o_arr = carve((size_t)max_rows * 4);
   const size_t o_st = carve(16);
@@ -222,6 +231,8 @@ IDX_API int idx_init(idx_ctx** out, int device, int max_rows, int max_n, int max
   ctx->ws = base;
   ctx->cand_bits = reinterpret_cast<uint32_t*>(base + o_bits);
   ctx->cand_idx = reinterpret_cast<int32_t*>(base + o_idx);
+  ctx->fcand_bits = reinterpret_cast<uint32_t*>(base + o_fbits);
+  ctx->fcand_idx = reinterpret_cast<int32_t*>(base + o_fidx);
   ctx->row_thr = reinterpret_cast<unsigned long long*>(base + o_thr);
   ctx->arrive = reinterpret_cast<int32_t*>(base + o_arr);
   ctx->status = reinterpret_cast<int*>(base + o_st);
@@ -319,13 +330,13 @@ static int fused_impl(idx_ctx* ctx, const uint16_t* q, const uint16_t* c,
       a.K = K;
       a.idx_out = idx_out + (int64_t)b0 * T * K;
       a.val_out = val_out ? val_out + (int64_t)b0 * T * K : nullptr;
-      a.cand_bits = ctx->cand_bits;
-      a.cand_idx = ctx->cand_idx;
+      a.cand_bits = ctx->fcand_bits;
+      a.cand_idx = ctx->fcand_idx;
       a.row_thr = ctx->row_thr;
-      a.slot_stride = ctx->max_k;
+      a.slot_stride = ctx->fused_stride;
       a.arrive = ctx->arrive;
       a.status = ctx->status;
-      if (idx::decode_fused_slots(nb, T, N, idx::decode_grid(ctx->num_sms)) > ctx->cand_slots)
+      if (idx::decode_fused_slots(nb, T, N, idx::decode_grid(ctx->num_sms)) > ctx->fused_slots)
         return IDX_ENOWORKSPACE;
       rc = status_of(idx::launch_decode(a, true, ctx->num_sms, st));
       if (rc != IDX_OK) return rc;

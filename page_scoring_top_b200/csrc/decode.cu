@@ -292,7 +292,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
     for (int b = ch.row(cb); b <= b_last; ++b) {
       if (ch.len(b) == 0) continue;
       const int p0 = ch.snap(b, cb);
-      const int np = ch.snap(b, ce) - p0;  // may be 0
+      const int np = ch.snap(b, ce) - p0;
+      if (np <= 0) continue;  // no real page of b in this chunk: not a segment
       if (FUSED) {
         fused_begin<HIST>(fsel, T);
         group_sync(kConsumers);

@@ -314,6 +314,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (ch.len(b) == 0) continue;
         const int p0 = ch.snap(b, cb);
         const int nps = ch.snap(b, ce) - p0;
+        if (nps <= 0) continue;  // no real page of b in this chunk: not a segment
         if (FUSED) {
           fused_begin<HIST>(fsel, T);
           group_sync(kTcEpi);

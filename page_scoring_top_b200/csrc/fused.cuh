@@ -12,6 +12,7 @@
 // "Iterate Centroids Score"; the tie rule of "Round 18 Track C", section 2.
 #pragma once
 
+#include "fsel.cuh"
 #include "hsel.cuh"
 #include "kernels.h"
 
@@ -113,57 +114,125 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
                                int j1) {
   SelectScratch& sc = *f.sc;
   if (HIST) {
-    // One token per row: the filter histogram is exact for the buffer, so one
-    // scan finds the boundary bin and the winners are placed from registers.
+    // One token per row.  The filter's digit histogram is exact for its
+    // buffer: one warp reads from it the digit b0 of the segment's K-th
+    // largest entry, so every entry of the segment's top K is >= vlo = b0's
+    // floor.  A segment that holds its whole request takes the exact ordered
+    // top K above vlo from registers (fine select, fsel.cuh).  Otherwise it
+    // publishes every entry >= vlo, unordered (about K plus one digit bin's
+    // worth), raises the request's threshold to vlo, and the last segment to
+    // arrive runs the fine select over all published entries.
     FilterState& fs = f.fst[0];
     uint32_t* fb = f.fbuf;
     uint32_t* fi = f.fbuf + f.cap;
-    uint32_t* start = &sc.hist[0][0];  // kHBins words
-    // boundary-bin members go to the front of the buffer once it is in registers
-    uint64_t* bl_v = reinterpret_cast<uint64_t*>(f.fbuf);
-    uint32_t* bl_b = f.fbuf + 2 * (kBoundaryMax + 2);
     const bool single = j0 == j1;
+    const int nslots = j1 - j0 + 1;
     int32_t* out_i = a.idx_out + (int64_t)b * a.K;
     float* out_v = a.val_out ? a.val_out + (int64_t)b * a.K : nullptr;
     const int64_t slot = (int64_t)(j + b);
-    hist_scan<kSelThreads>(f.hist, start, (uint32_t)a.K, sc);
+    uint32_t* cbits = a.cand_bits + slot * a.slot_stride;
+    int32_t* cidx = a.cand_idx + slot * a.slot_stride;
+    unsigned long long* row_thr = a.row_thr + b;
+    // Entries per published list: as many as the merge can hold in registers
+    // (kFilterCap over all lists), at least K, at most a slot, a multiple of 4
+    // (lists are copied 16 bytes at a time).
+    const int lcap = max((a.K + 3) & ~3, min((int)a.slot_stride, kFilterCap / nslots) & ~3);
+    // The areas: the fine histogram and its bin offsets in the second radix
+    // histogram of the scratch, the winners in the sort staging, the boundary
+    // list at the front of the buffer once the buffer is in registers.
+    uint32_t* fine = &sc.hist[1][0];
+    const FineArea ar{fine,    fine + kFineBins, f.sortv, f.sortb,
+                      reinterpret_cast<uint64_t*>(f.fbuf), f.fbuf + 2 * (kFineBoundaryMax + 2),
+                      sc.wsum, sc.bcast};
+    constexpr int E = kFilterCap / kSelThreads;
+    uint64_t v[E];
+    uint32_t bits[E];
+    auto out_emit = [&](int pos, uint64_t x, uint32_t xb) {
+      out_i[pos] = (int32_t)~(uint32_t)x;
+      if (out_v) out_v[pos] = __uint_as_float(xb);
+    };
+    auto out_pad = [&](int pos) {
+      out_i[pos] = -1;
+      if (out_v) out_v[pos] = __uint_as_float(kNegInfBits);
+    };
+    if ((threadIdx.x >> 5) == 0) warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)a.K, sc.bcast);
+    if (threadIdx.x == 0) sc.ctr = 0;
+    if (single) fine_clear<kSelThreads>(ar);
+    const int nk = load_buffer<kSelThreads, E>(fb, fi, fs.count, v, bits);
+    IDX_TRACE(19);
+    group_sync(kSelThreads);
+    const uint32_t b0 = sc.bcast[0], bmax = sc.bcast[1], n0 = sc.bcast[2];
+    const uint64_t vlo = (uint64_t)b0 << (32 + kHShift);
     IDX_TRACE(13);
-    if (sc.bcast[0] == 0xFFFFFFFFu || sc.bcast[2] <= (uint32_t)kBoundaryMax) {
-      constexpr int E = kFilterCap / kSelThreads;
-      uint64_t v[E];
-      uint32_t bits[E];
-      const int nk = load_buffer<kSelThreads, E>(fb, fi, fs.count, v, bits);
-      group_sync(kSelThreads);
-      if (single)
-        place_ordered<kSelThreads, E>(v, bits, nk, f.hist, start, a.K, sc, f.sortv, f.sortb, bl_v,
-                                      bl_b, out_i, out_v);
-      else
-        place_publish<kSelThreads, E>(v, bits, nk, start, a.K, sc, bl_v, bl_b,
-                                      a.cand_bits + slot * a.slot_stride,
-                                      a.cand_idx + slot * a.slot_stride, a.row_thr + b);
+    bool ok = true;
+    if (single) {
+      const uint32_t khi =
+          bmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((bmax + 1) << kHShift) - 1u;
+      ok = fine_select<kSelThreads, E>(v, bits, nk, vlo, khi, a.K, ar, out_emit, out_pad);
+    } else if (n0 <= (uint32_t)lcap) {
+#pragma unroll
+      for (int k = 0; k < E; ++k)
+        if (k < nk && v[k] >= vlo && v[k] != 0) {
+          const int p = atomicAdd(&sc.ctr, 1);
+          cbits[p] = bits[k];
+          cidx[p] = (int32_t)~(uint32_t)v[k];
+        }
+      for (int p = (int)n0 + (int)threadIdx.x; p < lcap; p += kSelThreads) {
+        cbits[p] = kNegInfBits;
+        cidx[p] = -1;
+      }
+      // with b0 > 0 the segment holds K entries >= vlo: so does its row
+      if (threadIdx.x == 0 && b0 != 0) atomicMax(row_thr, (unsigned long long)vlo);
     } else {
-      // a crowded boundary bin (heavy ties): radix compaction, then a plain write
+      ok = false;
+    }
+    if (!ok) {
+      // a crowded digit bin (heavy ties): exact radix compaction first
+      group_sync(kSelThreads);
       filter_compact<kSelThreads>(fs, fb, fi, a.K, sc);
-      if (single)
+      if (single) {
         sort_and_write<kSelThreads>(fb, fi, fs.count, a.K, f.sortv, f.sortb, out_i, out_v);
-      else
-        publish_candidates<kSelThreads>(fb, fi, fs.count, a.K, fs.thr,
-                                        a.cand_bits + slot * a.slot_stride,
-                                        a.cand_idx + slot * a.slot_stride, a.row_thr + b);
+      } else {
+        publish_candidates<kSelThreads>(fb, fi, fs.count, a.K, fs.thr, cbits, cidx, row_thr);
+        for (int p = a.K + (int)threadIdx.x; p < lcap; p += kSelThreads) {
+          cbits[p] = kNegInfBits;
+          cidx[p] = -1;
+        }
+      }
     }
     IDX_TRACE(14);
-    if (!single && arrive_last<kSelThreads>(a.arrive + b, j1 - j0 + 1, f.s_flag)) {
+    if (!single && arrive_last<kSelThreads>(a.arrive + b, nslots, f.s_flag)) {
       IDX_TRACE(15);
-      const int nslots = j1 - j0 + 1;
       auto slot_of = [=](int i) { return (int64_t)(j0 + i + b); };
       bool done = false;
-      if (nslots * a.K <= kFilterCap)
-        done = hist_merge_regs<kSelThreads, kFilterCap / kSelThreads>(
-            nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride, a.K, a.row_thr + b, f.hist,
-            start, sc, f.sortv, f.sortb, bl_v, bl_b, out_i, out_v);
+      if (nslots * lcap <= kFilterCap) {
+        // the buffer (already published) receives every list
+        stage_lists<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride, lcap,
+                                 fb, fi);
+        IDX_TRACE(25);
+        const int nkm = load_buffer<kSelThreads, E>(fb, fi, nslots * lcap, v, bits);
+        uint32_t km = 0;
+#pragma unroll
+        for (int k = 0; k < E; ++k) km = max(km, (uint32_t)(v[k] >> 32));
+        km = __reduce_max_sync(0xFFFFFFFFu, km);
+        if (lane_id() == 0) sc.wsum[threadIdx.x >> 5] = km;
+        if (threadIdx.x == 0) {
+          *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = __ldcg(row_thr);
+          *row_thr = 0ull;  // zero for the next call
+        }
+        fine_clear<kSelThreads>(ar);
+        group_sync(kSelThreads);
+        IDX_TRACE(26);
+        const uint64_t thr = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
+        km = 0;
+#pragma unroll
+        for (int w = 0; w < kSelThreads / 32; ++w) km = max(km, sc.wsum[w]);
+        done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, a.K, ar, out_emit, out_pad);
+        if (!done) group_sync(kSelThreads);
+      }
       if (!done)
         merge_candidates<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride,
-                                      a.K, a.row_thr + b, fs, f.fbuf, f.fbuf + kFilterCap,
+                                      lcap, a.K, row_thr, fs, f.fbuf, f.fbuf + kFilterCap,
                                       kFilterCap, sc, f.sortv, f.sortb, out_i, out_v);
       IDX_TRACE(16);
     }
@@ -189,7 +258,7 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
         const int64_t orow = (int64_t)b * T + t;
         merge_candidates<kSelThreads>(
             j1 - j0 + 1, [=](int i) { return (int64_t)(j0 + i + b) * T + t; }, a.cand_bits,
-            a.cand_idx, a.slot_stride, a.K, a.row_thr + orow, f.fst[0], f.fbuf,
+            a.cand_idx, a.slot_stride, a.K, a.K, a.row_thr + orow, f.fst[0], f.fbuf,
             f.fbuf + kFilterCap, kFilterCap, sc, f.sortv, f.sortb, a.idx_out + orow * a.K,
             a.val_out ? a.val_out + orow * a.K : nullptr);
       }
@@ -311,8 +380,15 @@ struct Chunking {
     if (r >= n) return n;
     return r <= 0 ? 0 : (r & ~31);
   }
-  // Chunks holding a segment of request b: first0(b) .. last(b).
-  __device__ __forceinline__ int first(int b) const { return voff(b) / Lc; }
+  // Chunks holding a segment of request b (a nonempty page range):
+  // first(b) .. last(b).  The chunk holding b's first real page may see
+  // fewer than 32 of them, which snap to none; its segment then starts in the
+  // next chunk.  With chunks of at least 64 pages every chunk in between
+  // holds a nonempty segment.
+  __device__ __forceinline__ int first(int b) const {
+    const int x = voff(b) + W + min(len(b), 32);  // first virtual end with a real page
+    return min((x - 1) / Lc, nchunks - 1);
+  }
   __device__ __forceinline__ int last(int b) const { return (voff(b + 1) - 1) / Lc; }
   __device__ __forceinline__ int chunk_begin(int j) const { return j * Lc; }
   __device__ __forceinline__ int chunk_end(int j) const { return min(j * Lc + Lc, PV); }

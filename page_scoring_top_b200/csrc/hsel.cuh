@@ -1,27 +1,20 @@
-// hsel.cuh -- exact top-K driven by a histogram of the candidates' top digits.
+// hsel.cuh -- the running digit histogram of an online top-K filter.
 //
 // A candidate's digit is the top 12 bits of its order key (sign, exponent and
 // three mantissa bits of the score: bins an eighth of an octave wide).  A
 // filter (select.cuh) that also keeps the histogram of its buffer -- one
 // shared-memory atomic per appended entry, plus one on a 128-bin coarse copy
-// (digit >> 5) -- gets three things cheaply:
-//  * a running threshold: the highest digit b with at least K buffered entries
-//    in bins >= b bounds the K-th largest value from below, so "keep digit >= b"
-//    is exact.  One warp reads it off the coarse and fine histograms in a few
-//    instructions, from a racy snapshot (counts only grow, so a snapshot
-//    under-counts, which keeps the bound valid), without stopping the others;
-//    the buffer then never needs a mid-stream compaction;
-//  * the winners in one pass: entries above bin b are winners, and the top
-//    r = K - (entries above b) of bin b are found by counting among that bin's
-//    few members;
-//  * the output order without a sort: a winner's position is the number of
-//    winners in higher bins plus its rank among the winners of its own bin.
-// Rank values (key << 32 | ~index) are unique, so ties need no extra rule.
-// A crowded boundary bin (heavy ties) or a buffer about to overflow falls back
-// to the radix compaction of select.cuh.  The digit histogram is the
-// radix-select machinery of "Iterate Topk" (radix family) and of qsa_topk2
-// ("Round 18 Track C", section 1 Target 1), kept as a running statistic of the
-// stream instead of recomputed in passes over the row.
+// (digit >> 5) -- gets a running threshold cheaply: the highest digit b with
+// at least K buffered entries in bins >= b bounds the K-th largest value from
+// below, so "keep digit >= b" is exact.  One lane reads it off the coarse and
+// fine histograms in a few instructions, from a racy snapshot (counts only
+// grow, so a snapshot under-counts, which keeps the bound valid), without
+// stopping the others; the buffer then rarely needs a compaction.  At the end
+// of a segment the same floor tells the fine select (fsel.cuh) where the top K
+// starts.  The digit histogram is the radix-select machinery of "Iterate Topk"
+// (radix family) and of qsa_topk2 ("Round 18 Track C", section 1 Target 1),
+// kept as a running statistic of the stream instead of recomputed in passes
+// over the row.
 #pragma once
 
 #include "select.cuh"
@@ -32,7 +25,6 @@ constexpr int kHBits = 12;
 constexpr int kHBins = 1 << kHBits;          // 4096 fine bins
 constexpr int kHShift = 32 - kHBits;         // digit = key >> kHShift
 constexpr int kHCoarse = kHBins / 32;        // 128 coarse bins of 32 fine bins
-constexpr int kBoundaryMax = 256;            // bin-b members resolved by counting
 
 __device__ __forceinline__ uint32_t hdigit_v(uint64_t v) {
   return (uint32_t)(v >> (32 + kHShift));
@@ -129,193 +121,6 @@ __device__ __forceinline__ void raise_threshold_1t(FilterState& fs, const uint32
   }
 }
 
-// Scan of an exact 4096-bin histogram (all NT threads, two barriers):
-// start[d] = entries in bins above d (exclusive suffix sum) and the top-K
-// boundary, broadcast as bcast[0] = b (the bin holding the K-th largest
-// entry; 0xFFFFFFFF when total <= K: every entry is a winner), bcast[1] =
-// entries above b, bcast[2] = hist[b], bcast[3] = total.  Each thread owns 16
-// consecutive bins (thread 0 the top ones), read and written 16 bytes at a time.
-template <int NT>
-__device__ __forceinline__ void hist_scan(const uint32_t* hist, uint32_t* start, uint32_t K,
-                                          SelectScratch& sc) {
-  constexpr int BPT = kHBins / NT;
-  static_assert(kHBins % NT == 0 && BPT % 4 == 0, "bins per thread");
-  const int tid = threadIdx.x;
-  const int lo = kHBins - (tid + 1) * BPT;
-  uint32_t h[BPT];
-#pragma unroll
-  for (int k = 0; k < BPT; k += 4) {
-    const uint4 q = *reinterpret_cast<const uint4*>(hist + lo + k);
-    h[k] = q.x;
-    h[k + 1] = q.y;
-    h[k + 2] = q.z;
-    h[k + 3] = q.w;
-  }
-  uint32_t s = 0;
-#pragma unroll
-  for (int k = 0; k < BPT; ++k) s += h[k];
-  const uint32_t incl = warp_incl_scan(s);
-  const int warp = tid >> 5;
-  if (lane_id() == 31) sc.wsum[warp] = incl;
-  group_sync(NT);
-  uint32_t excl = incl - s, total = 0;
-#pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    const uint32_t x = sc.wsum[w];
-    if (w < warp) excl += x;
-    total += x;
-  }
-  if (tid == 0) {
-    sc.bcast[3] = total;
-    if (total <= K) {
-      sc.bcast[0] = 0xFFFFFFFFu;
-      sc.bcast[1] = total;
-      sc.bcast[2] = 0u;
-    }
-  }
-  uint32_t st[BPT];
-  uint32_t cum = excl;
-  bool found = !(total > K && excl < K && K <= excl + s);
-#pragma unroll
-  for (int k = BPT - 1; k >= 0; --k) {
-    st[k] = cum;
-    if (!found && cum + h[k] >= K) {
-      sc.bcast[0] = (uint32_t)(lo + k);
-      sc.bcast[1] = cum;
-      sc.bcast[2] = h[k];
-      found = true;
-    }
-    cum += h[k];
-  }
-#pragma unroll
-  for (int k = 0; k < BPT; k += 4)
-    *reinterpret_cast<uint4*>(start + lo + k) = make_uint4(st[k], st[k + 1], st[k + 2], st[k + 3]);
-  group_sync(NT);
-}
-
-// Rank each of the cnt members of the boundary bin (bl_v / bl_b; bl_v holds
-// a zero after the last member, 16-byte aligned) among the others and hand
-// the r largest to sink(rank, v, bits).  One member per thread, compared
-// against all members two at a time (rank values are unique).
-template <int NT, class Sink>
-__device__ __forceinline__ void rank_boundary(const uint64_t* bl_v, const uint32_t* bl_b, int cnt,
-                                              int r, Sink sink) {
-  const int half = (cnt + 1) >> 1;
-  for (int t = threadIdx.x; t < cnt; t += NT) {
-    const uint64_t x = bl_v[t];
-    int rank = 0;
-#pragma unroll 4
-    for (int j = 0; j < half; ++j) {
-      const ulonglong2 u = reinterpret_cast<const ulonglong2*>(bl_v)[j];
-      rank += (u.x > x) + (u.y > x);
-    }
-    if (rank < r) sink(rank, x, bl_b[t]);
-  }
-}
-
-// Split register-held entries (v[k], bits[k] for k < nk; v = 0 marks none)
-// by the boundary bin b of hist_scan, taking positions from the start[]
-// counters that hist_scan left: an entry of a higher bin calls win(v, bits,
-// digit, slot) with slot = start[digit]++ (so the winners fill [0, above),
-// grouped by bin, highest bin first); a member of bin b is appended to the
-// bl list at start[b]++ - above.
-template <int E, class Win>
-__device__ __forceinline__ void classify(const uint64_t (&v)[E], const uint32_t (&bits)[E], int nk,
-                                         uint32_t b, uint32_t above, uint32_t* start,
-                                         uint64_t* bl_v, uint32_t* bl_b, Win win) {
-#pragma unroll
-  for (int k = 0; k < E; ++k) {
-    if (k >= nk) break;
-    if (v[k] == 0) continue;
-    const uint32_t d = hdigit_v(v[k]);
-    if (b == 0xFFFFFFFFu || d > b) {
-      win(v[k], bits[k], d, atomicAdd(&start[d], 1u));
-    } else if (d == b) {
-      const uint32_t p = atomicAdd(&start[d], 1u) - above;
-      bl_v[p] = v[k];
-      bl_b[p] = bits[k];
-    }
-  }
-}
-
-// Exact top K of register-held entries, written as one ordered output row.
-// hist must be the exact histogram of the entries and hist_scan must have run
-// on it (start, sc.bcast) with no boundary bin above kBoundaryMax.  A
-// winner's position = winners in higher bins + its rank among the winners of
-// its bin; the r largest members of bin b follow all of them.  tv/tb stage
-// the winners (K entries); bl_v/bl_b hold kBoundaryMax + 2.  Slots past
-// min(K, total) get -1 / -inf.
-template <int NT, int E>
-__device__ void place_ordered(const uint64_t (&v)[E], const uint32_t (&bits)[E], int nk,
-                              const uint32_t* hist, uint32_t* start, int K, SelectScratch& sc,
-                              uint64_t* tv, uint32_t* tb, uint64_t* bl_v, uint32_t* bl_b,
-                              int32_t* idx_out, float* val_out) {
-  const int tid = threadIdx.x;
-  const uint32_t b = sc.bcast[0];
-  const int above = (int)sc.bcast[1];
-  const int cnt = (int)sc.bcast[2];
-  const int total = (int)sc.bcast[3];
-  classify(v, bits, nk, b, (uint32_t)above, start, bl_v, bl_b,
-           [&](uint64_t x, uint32_t xb, uint32_t, uint32_t slot) {
-             tv[slot] = x;
-             tb[slot] = xb;
-           });
-  if (tid == 0) bl_v[cnt] = 0ull;
-  group_sync(NT);
-  // start[d] now ends bin d's range of tv
-  for (int i = tid; i < above; i += NT) {
-    const uint64_t x = tv[i];
-    const uint32_t d = hdigit_v(x);
-    const int hi = (int)start[d];
-    int pos = hi - (int)hist[d];
-    for (int j = pos; j < hi; ++j) pos += tv[j] > x;
-    idx_out[pos] = (int32_t)~(uint32_t)x;
-    if (val_out) val_out[pos] = __uint_as_float(tb[i]);
-  }
-  rank_boundary<NT>(bl_v, bl_b, cnt, K - above, [&](int rank, uint64_t x, uint32_t xb) {
-    idx_out[above + rank] = (int32_t)~(uint32_t)x;
-    if (val_out) val_out[above + rank] = __uint_as_float(xb);
-  });
-  for (int k = min(total, K) + tid; k < K; k += NT) {
-    idx_out[k] = -1;
-    if (val_out) val_out[k] = __uint_as_float(kNegInfBits);
-  }
-  group_sync(NT);
-}
-
-// Exact top K of register-held entries as one unordered candidate list of
-// exactly K entries (cbits / cidx; unused entries -inf / -1), after
-// hist_scan on their exact histogram.  When entries were dropped, the K-th
-// largest rank value raises *row_thr (atomic max): every entry of the row's
-// top K is at least that.
-template <int NT, int E>
-__device__ void place_publish(const uint64_t (&v)[E], const uint32_t (&bits)[E], int nk,
-                              uint32_t* start, int K, SelectScratch& sc, uint64_t* bl_v,
-                              uint32_t* bl_b, uint32_t* cbits, int32_t* cidx,
-                              unsigned long long* row_thr) {
-  const uint32_t b = sc.bcast[0];
-  const int above = (int)sc.bcast[1];
-  const int cnt = (int)sc.bcast[2];
-  const int total = (int)sc.bcast[3];
-  classify(v, bits, nk, b, (uint32_t)above, start, bl_v, bl_b,
-           [&](uint64_t x, uint32_t xb, uint32_t, uint32_t slot) {
-             cbits[slot] = xb;
-             cidx[slot] = (int32_t)~(uint32_t)x;
-           });
-  if (threadIdx.x == 0) bl_v[cnt] = 0ull;
-  group_sync(NT);
-  const int r = K - above;
-  rank_boundary<NT>(bl_v, bl_b, cnt, r, [&](int rank, uint64_t x, uint32_t xb) {
-    cbits[above + rank] = xb;
-    cidx[above + rank] = (int32_t)~(uint32_t)x;
-    if (rank == r - 1) atomicMax(row_thr, (unsigned long long)x);
-  });
-  for (int k = min(total, K) + (int)threadIdx.x; k < K; k += NT) {
-    cbits[k] = kNegInfBits;
-    cidx[k] = -1;
-  }
-}
-
 // Load a filter buffer's n entries into registers (entry i = tid + k * NT).
 template <int NT, int E>
 __device__ __forceinline__ int load_buffer(const uint32_t* fb, const uint32_t* fi, int n,
@@ -332,66 +137,6 @@ __device__ __forceinline__ int load_buffer(const uint32_t* fb, const uint32_t* f
     }
   }
   return nk;
-}
-
-// Merge published candidate lists (list i at bits/index + slot_of(i) *
-// stride, K entries each, unused entries -inf) into one ordered output row,
-// when all nslots * K entries fit in registers (E per thread).  Every thread
-// issues all its loads at once (the row threshold is read meanwhile);
-// entries below the threshold are dropped, the rest counted in hist, and the
-// exact winners are placed in order.  Resets *row_thr to zero for the next
-// call.  Returns false, having done nothing but the reset, when the boundary
-// bin is too crowded (heavy ties): the caller then merges another way.
-template <int NT, int E, class SlotOf>
-__device__ bool hist_merge_regs(int nslots, SlotOf slot_of, const uint32_t* cand_bits,
-                                const int32_t* cand_idx, int64_t stride, int K,
-                                unsigned long long* row_thr, uint32_t* hist, uint32_t* start,
-                                SelectScratch& sc, uint64_t* tv, uint32_t* tb, uint64_t* bl_v,
-                                uint32_t* bl_b, int32_t* idx_out, float* val_out) {
-  const int tid = threadIdx.x;
-  const int total = nslots * K;
-  uint64_t v[E];
-  uint32_t bits[E];
-  uint32_t index[E];
-  int i0 = tid / K, e0 = tid - i0 * K;  // list and entry of f = tid, advanced by NT
-  const int di = NT / K, de = NT - di * K;
-#pragma unroll
-  for (int k = 0; k < E; ++k) {
-    bits[k] = kNegInfBits;
-    index[k] = 0u;
-    if (k * NT + tid < total) {
-      const int64_t off = slot_of(i0) * stride + e0;
-      bits[k] = __ldcg(cand_bits + off);
-      index[k] = (uint32_t)__ldcg(cand_idx + off);
-    }
-    i0 += di;
-    e0 += de;
-    if (e0 >= K) {
-      e0 -= K;
-      ++i0;
-    }
-  }
-  for (int i = tid; i < kHBins; i += NT) hist[i] = 0u;
-  if (tid == 0) {
-    const unsigned long long t = __ldcg(row_thr);
-    *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = t ? t - 1 : 0ull;  // keep v >= t
-    *row_thr = 0ull;
-  }
-  group_sync(NT);
-  const unsigned long long thr = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
-  int nk = 0;
-#pragma unroll
-  for (int k = 0; k < E; ++k) {
-    const uint64_t x = rank_value(bits[k], index[k]);
-    v[k] = x > thr ? x : 0ull;
-    if (v[k]) atomicAdd(&hist[hdigit_v(v[k])], 1u);
-    if (k * NT < total) nk = k + 1;
-  }
-  group_sync(NT);
-  hist_scan<NT>(hist, start, (uint32_t)K, sc);
-  if (sc.bcast[0] != 0xFFFFFFFFu && sc.bcast[2] > (uint32_t)kBoundaryMax) return false;
-  place_ordered<NT, E>(v, bits, nk, hist, start, K, sc, tv, tb, bl_v, bl_b, idx_out, val_out);
-  return true;
 }
 
 }  // namespace idx

@@ -386,14 +386,14 @@ __device__ void publish_candidates(const uint32_t* fb, const uint32_t* fi, int k
 }
 
 // Merge nslots published lists (list i at bits/index + slot_of(i) * stride,
-// K entries each) into one final row.  All lists are fetched with every
+// L entries each, unused entries invalid) into one final row of K.  All lists are fetched with every
 // thread's loads in flight together; entries below the row threshold are
 // dropped on arrival; the survivors are placed by the counting sort when few
 // enough remain, else compacted first.  Resets *row_thr to zero for the next
 // call.  fb/fi is a filter buffer of cap >= K + NT * 8 entries.
 template <int NT, class SlotOf>
 __device__ void merge_candidates(int nslots, SlotOf slot_of, const uint32_t* cand_bits,
-                                 const int32_t* cand_idx, int64_t stride, int K,
+                                 const int32_t* cand_idx, int64_t stride, int L, int K,
                                  unsigned long long* row_thr, FilterState& fs, uint32_t* fb,
                                  uint32_t* fi, int cap, SelectScratch& sc, uint64_t* sv,
                                  uint32_t* sb, int32_t* idx_out, float* val_out) {
@@ -407,7 +407,7 @@ __device__ void merge_candidates(int nslots, SlotOf slot_of, const uint32_t* can
     *row_thr = 0ull;
   }
   group_sync(NT);
-  const int total = nslots * K;
+  const int total = nslots * L;
   for (int f0 = 0; f0 < total; f0 += NT * U) {
     uint32_t bits[U], index[U];
 #pragma unroll
@@ -416,8 +416,8 @@ __device__ void merge_candidates(int nslots, SlotOf slot_of, const uint32_t* can
       bits[u] = kNegInfBits;
       index[u] = 0xFFFFFFFFu;
       if (f < total) {
-        const int i = f / K;
-        const int e = f - i * K;
+        const int i = f / L;
+        const int e = f - i * L;
         const int64_t off = slot_of(i) * stride + e;
         bits[u] = __ldcg(cand_bits + off);
         index[u] = (uint32_t)__ldcg(cand_idx + off);
@@ -441,20 +441,19 @@ __device__ void merge_candidates(int nslots, SlotOf slot_of, const uint32_t* can
 // All threads of the group: count one arrival on *counter once this CTA's
 // global stores are visible GPU-wide.  Returns true (to every thread) in the
 // CTA that arrives last (the expected-th arrival), which also resets the
-// counter to zero; its reads of the other CTAs' stores are ordered after
-// theirs.  The barrier orders every thread's stores before thread 0's
-// release fence and arrival; thread 0's acquire fence and the second barrier
-// order the other CTAs' stores before this CTA's later reads.
+// counter to zero.  The barrier orders every thread's stores before thread
+// 0's arrival, a GPU-scope acquire-release atomic: its release half publishes
+// them (release is cumulative over what the barrier ordered before it), its
+// acquire half orders the other CTAs' published stores before this CTA's
+// later reads, which the second barrier extends to every thread.
 template <int NT>
 __device__ bool arrive_last(int32_t* counter, int expected, int* s_flag) {
   group_sync(NT);
   if (threadIdx.x == 0) {
-    __threadfence();
-    const bool last = atomicAdd(counter, 1) == expected - 1;
-    if (last) {
-      *counter = 0;
-      __threadfence();
-    }
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(old) : "l"(counter) : "memory");
+    const bool last = old == expected - 1;
+    if (last) *counter = 0;  // no CTA of this launch touches it again
     *s_flag = last;
   }
   group_sync(NT);

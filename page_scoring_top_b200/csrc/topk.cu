@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(NT) topk_chunk_kernel(const TopkArgs a) {
   if (!arrive_last<NT>(a.arrive + row, nch, s_flag)) return;
   const int64_t base = (int64_t)row * a.max_chunks;
   merge_candidates<NT>(
-      nch, [base](int i) { return base + i; }, a.cand_bits, a.cand_idx, a.slot_stride, a.K,
+      nch, [base](int i) { return base + i; }, a.cand_bits, a.cand_idx, a.slot_stride, a.K, a.K,
       a.row_thr + row, fs, fb, fi, kFilterCap, sc, sortv, sortb, io, vo);
 }
 
