@@ -138,7 +138,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   int* misc = reinterpret_cast<int*>(smem + L.misc);
   volatile int* s_abort = misc;
   uint32_t* s_wsum = reinterpret_cast<uint32_t*>(misc + 4);  // 9 warp sums
-  const FusedSel fsel{fbuf, fst, &sc, sortv, sortb, hist, L.cap, misc + 1};
+  const FusedSel fsel{fbuf, fst,   &sc,    sortv, sortb, hist, L.cap, misc + 1,
+                      reinterpret_cast<uint32_t*>(misc + 14)};
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
           if (lane == 0) mbar_arrive(&empty[slot]);
           // Every fourth of its stages, a warp lifts the threshold to the
           // histogram's top-K bin; two warps of each round do it.
-          if (HIST && ((stage >> 3) & 3) == (uint32_t)(warp & 3)) fused_raise(fsel, a.K);
+          if (HIST && ((stage >> 3) & 3) == (uint32_t)(warp & 3)) fused_raise(fsel, a.K, a.row_thr + b);
         }
         if (FUSED && ((stage % check_period) == check_period - 1 || sp + kStagePages >= np)) {
           group_sync(kConsumers);  // this round's offers are complete

@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       reinterpret_cast<uint32_t*>(smem + L.sortb),
                       reinterpret_cast<uint32_t*>(smem + L.hist),
                       L.cap,
-                      misc + 1};
+                      misc + 1,
+                      reinterpret_cast<uint32_t*>(misc + 14)};
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, g = blockIdx.x;
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // twice per 8 tiles (once per warpgroup), one warp lifts the
             // threshold from the histogram
             if (HIST && (tile & 7) == (wg ? 5u : 0u) && (int)((tile >> 3) & 3) == quad)
-              fused_raise(fsel, a.K);
+              fused_raise(fsel, a.K, a.row_thr + b);
           }
           if (FUSED && (tt == next_check || tt + 1 == ntl)) {
             group_sync(kTcEpi);  // every offer so far is complete

@@ -179,10 +179,11 @@ __device__ bool fine_select(const uint64_t (&v)[E], const uint32_t (&bits)[E], i
 // histogram (hsel.cuh: hist kHBins words, chist kHCoarse words), computed by
 // one whole warp: out[0] = the digit holding the K-th largest entry (0 when
 // fewer than K entries), out[1] = the highest nonzero digit (0 when empty),
-// out[2] = the number of entries with digit >= out[0].  Every entry of the
+// out[3] = max(out[0], dmin) (a floor raised by a bound known from elsewhere),
+// out[2] = the number of entries with digit >= out[3].  Every entry of the
 // buffer's top K then has digit >= out[0], and every entry has digit <= out[1].
 __device__ __forceinline__ void warp_hist_bounds(const uint32_t* hist, const uint32_t* chist,
-                                                 uint32_t K, uint32_t* out) {
+                                                 uint32_t K, uint32_t dmin, uint32_t* out) {
   const uint32_t lane = lane_id();
   // coarse bins, lane l owning 4(31 - l) .. 4(31 - l) + 3 (lane 0 the top)
   const uint4 q = reinterpret_cast<const uint4*>(chist)[31 - lane];
@@ -226,10 +227,22 @@ __device__ __forceinline__ void warp_hist_bounds(const uint32_t* hist, const uin
     b0 = 32 * cb + 31 - (__ffs(fh) - 1);
     n0 = __shfl_sync(0xFFFFFFFFu, fi, __ffs(fh) - 1);
   }
+  if (dmin > b0) {
+    // entries at or above dmin: coarse bins above its own, then its fine bins
+    const uint32_t cd = dmin >> 5;
+    uint32_t part = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (4 * (31 - lane) + 3 - e > cd) part += ch[e];
+    const uint32_t f = hist[32 * cd + 31 - lane];
+    if (31 - lane >= (dmin & 31)) part += f;
+    n0 = __reduce_add_sync(0xFFFFFFFFu, part);
+  }
   if (lane == 0) {
     out[0] = b0;
     out[1] = bmax;
     out[2] = n0;
+    out[3] = max(b0, dmin);
   }
 }
 

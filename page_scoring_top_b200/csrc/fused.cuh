@@ -35,6 +35,9 @@ struct FusedSel {
   uint32_t* hist;       // kHBins + kHCoarse words (single-token rows only)
   int cap;              // filter entries per token
   int* s_flag;
+  // single-token rows: the last polled high word of the request's shared
+  // threshold (its key part), copied in asynchronously while streaming
+  uint32_t* s_row;
 };
 
 // Filter entries per token for T tokens.
@@ -48,7 +51,10 @@ __host__ __device__ inline int fused_cap(int T) {
 template <bool HIST>
 __device__ __forceinline__ void fused_begin(const FusedSel& f, int T) {
   if ((int)threadIdx.x < T) filter_reset(f.fst[threadIdx.x]);
-  if (HIST) hist_clear<kSelThreads>(f.hist, f.hist + kHBins);
+  if (HIST) {
+    hist_clear<kSelThreads>(f.hist, f.hist + kHBins);
+    if (threadIdx.x == 0) *f.s_row = 0u;
+  }
 }
 
 // One warp offers its 32 lanes' scores of token t.
@@ -64,9 +70,28 @@ __device__ __forceinline__ void fused_offer(const FusedSel& f, int t, uint32_t b
 }
 
 // Lane 0 of the calling warp lifts the single-token filter's threshold from
-// its histogram.
-__device__ __forceinline__ void fused_raise(const FusedSel& f, int K) {
-  if (lane_id() == 0) raise_threshold_1t(f.fst[0], f.hist, f.hist + kHBins, K);
+// its histogram, and shares it with the other CTAs streaming the same
+// request: the filter's floor raises the request's threshold *row_thr
+// (atomic max; a segment's K-th largest bounds its request's from below),
+// and the request's threshold as last polled raises the filter's, so a
+// segment stops buffering what another segment has already beaten.  The poll
+// is an asynchronous 4-byte copy of the threshold's key half into s_row,
+// read at the next raise: never a stall on global memory.
+__device__ __forceinline__ void fused_raise(const FusedSel& f, int K,
+                                            unsigned long long* row_thr) {
+  if (lane_id() != 0) return;
+  FilterState& fs = f.fst[0];
+  const uint32_t b = hist_floor_1t(f.hist, f.hist + kHBins, (uint32_t)K);
+  unsigned long long t = fs.thr;
+  if (b != 0u) {
+    const unsigned long long fl = (unsigned long long)b << (32 + kHShift);
+    t = max(t, fl - 1ull);
+    atomicMax(row_thr, fl);
+  }
+  const uint32_t hi = *reinterpret_cast<volatile uint32_t*>(f.s_row);
+  if (hi != 0u) t = max(t, ((unsigned long long)hi << 32) - 1ull);
+  if (t > fs.thr) fs.thr = t;
+  cp_async4(f.s_row, reinterpret_cast<const uint32_t*>(row_thr) + 1);
 }
 
 // Overflow guard at a check point (all select threads, after a barrier that
@@ -155,14 +180,25 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
       out_i[pos] = -1;
       if (out_v) out_v[pos] = __uint_as_float(kNegInfBits);
     };
-    if ((threadIdx.x >> 5) == 0) warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)a.K, sc.bcast);
-    if (threadIdx.x == 0) sc.ctr = 0;
+    // Every asynchronous poll of the request's threshold has landed (the
+    // next segment may belong to another request).
+    cp_async_wait_all();
+    if ((threadIdx.x >> 5) == 0)
+      warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)a.K, single ? 0u : *f.s_row >> kHShift,
+                       sc.bcast);
+    if (threadIdx.x == 0) {
+      sc.ctr = 0;
+      if (single) *row_thr = 0ull;  // raised while streaming, read by nobody else
+    }
     if (single) fine_clear<kSelThreads>(ar);
     const int nk = load_buffer<kSelThreads, E>(fb, fi, fs.count, v, bits);
     IDX_TRACE(19);
     group_sync(kSelThreads);
-    const uint32_t b0 = sc.bcast[0], bmax = sc.bcast[1], n0 = sc.bcast[2];
+    // b0: the digit of the segment's K-th largest; bp >= b0: the publish
+    // floor, raised to the request's threshold; n0: entries at or above bp.
+    const uint32_t b0 = sc.bcast[0], bmax = sc.bcast[1], n0 = sc.bcast[2], bp = sc.bcast[3];
     const uint64_t vlo = (uint64_t)b0 << (32 + kHShift);
+    const uint64_t vpub = (uint64_t)bp << (32 + kHShift);
     IDX_TRACE(13);
     bool ok = true;
     if (single) {
@@ -172,7 +208,7 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
     } else if (n0 <= (uint32_t)lcap) {
 #pragma unroll
       for (int k = 0; k < E; ++k)
-        if (k < nk && v[k] >= vlo && v[k] != 0) {
+        if (k < nk && v[k] >= vpub && v[k] != 0) {
           const int p = atomicAdd(&sc.ctr, 1);
           cbits[p] = bits[k];
           cidx[p] = (int32_t)~(uint32_t)v[k];
@@ -228,7 +264,28 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
 #pragma unroll
         for (int w = 0; w < kSelThreads / 32; ++w) km = max(km, sc.wsum[w]);
         done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, a.K, ar, out_emit, out_pad);
-        if (!done) group_sync(kSelThreads);
+        if (!done) {
+          // a crowded boundary bin (heavy ties): the entries at or above the
+          // threshold go back to the buffer for the exact radix compaction
+          if (threadIdx.x == 0) sc.ctr = 0;
+          group_sync(kSelThreads);
+#pragma unroll
+          for (int k = 0; k < E; ++k)
+            if (k < nkm && v[k] >= thr && v[k] != 0) {
+              const int p = atomicAdd(&sc.ctr, 1);
+              fb[p] = bits[k];
+              fi[p] = ~(uint32_t)v[k];
+            }
+          group_sync(kSelThreads);
+          if (threadIdx.x == 0) {
+            fs.count = sc.ctr;
+            fs.thr = 0ull;
+          }
+          group_sync(kSelThreads);
+          filter_compact<kSelThreads>(fs, fb, fi, a.K, sc);
+          sort_and_write<kSelThreads>(fb, fi, fs.count, a.K, f.sortv, f.sortb, out_i, out_v);
+          done = true;
+        }
       }
       if (!done)
         merge_candidates<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride,
