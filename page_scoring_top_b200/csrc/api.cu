@@ -80,6 +80,36 @@ int status_of(cudaError_t e) { return e == cudaSuccess ? IDX_OK : IDX_ECUDA; }
 
 int run_topk(idx_ctx* ctx, const float* scores, const int32_t* lengths, int len_div, int rows,
              int N, int64_t lds, int K, int32_t* idx_out, float* val_out, cudaStream_t stream) {
+  if (idx::topk_stream_supported(scores, lds)) {
+    // the streamed kernel, in blocks of rows; its candidate slots are the
+    // fused path's (chunk + row per launch)
+    // (a block is a whole number of length groups: rows r use lengths[r / len_div])
+    const int rmax = std::max(1, idx::topk_stream_max_rows() / len_div) * len_div;
+    if (rmax > idx::topk_stream_max_rows()) return IDX_EUNSUPPORTED;
+    for (int r0 = 0; r0 < rows; r0 += rmax) {
+      const int nr = std::min(rmax, rows - r0);
+      if (idx::topk_stream_slots(nr, ctx->num_sms) > ctx->fused_slots) return IDX_ENOWORKSPACE;
+      idx::TopkStreamArgs s{};
+      s.scores = scores + (int64_t)r0 * lds;
+      s.lengths = lengths ? lengths + r0 / len_div : nullptr;
+      s.len_div = len_div;
+      s.rows = nr;
+      s.N = N;
+      s.lds = lds;
+      s.K = K;
+      s.idx_out = idx_out + (int64_t)r0 * K;
+      s.val_out = val_out ? val_out + (int64_t)r0 * K : nullptr;
+      s.cand_bits = ctx->fcand_bits;
+      s.cand_idx = ctx->fcand_idx;
+      s.slot_stride = ctx->fused_stride;
+      s.row_thr = ctx->row_thr + r0;
+      s.arrive = ctx->arrive + r0;
+      s.status = ctx->status;
+      const int rc = status_of(idx::launch_topk_stream(s, ctx->num_sms, stream));
+      if (rc != IDX_OK) return rc;
+    }
+    return IDX_OK;
+  }
   idx::TopkArgs a{};
   a.scores = scores;
   a.lengths = lengths;

@@ -119,6 +119,34 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+// Non-blocking test of phase `parity` of `bar`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait_bounded for a group of warps that all wait for the same phase and
+// then meet at a barrier: a spin on the non-blocking test, so that no warp
+// sleeps past the phase's completion (the slowest waker would hold up the
+// whole group).  The same iteration limit and abort protocol.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort, int* status) {
+  for (uint32_t it = 0; it < 4u * kMaxWaitIters; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (*abort) return false;
+  }
+  *abort = 1;
+  atomicOr(status, kErrWaitTimeout);
+  return false;
+}
+
 // Bounded wait that ignores the abort flag: a producer draining its own copies
 // in flight before the CTA exits.
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {

@@ -69,8 +69,8 @@ __device__ __forceinline__ void fused_offer(const FusedSel& f, int t, uint32_t b
   }
 }
 
-// Lane 0 of the calling warp lifts the single-token filter's threshold from
-// its histogram, and shares it with the other CTAs streaming the same
+// The calling warp (all lanes) reads the floor off the histogram, then lane 0
+// lifts the single-token filter's threshold to it, and shares it with the other CTAs streaming the same
 // request: the filter's floor raises the request's threshold *row_thr
 // (atomic max; a segment's K-th largest bounds its request's from below),
 // and the request's threshold as last polled raises the filter's, so a
@@ -79,9 +79,9 @@ __device__ __forceinline__ void fused_offer(const FusedSel& f, int t, uint32_t b
 // read at the next raise: never a stall on global memory.
 __device__ __forceinline__ void fused_raise(const FusedSel& f, int K,
                                             unsigned long long* row_thr) {
+  const uint32_t b = hist_floor_warp(f.hist, f.hist + kHBins, (uint32_t)K);
   if (lane_id() != 0) return;
   FilterState& fs = f.fst[0];
-  const uint32_t b = hist_floor_1t(f.hist, f.hist + kHBins, (uint32_t)K);
   unsigned long long t = fs.thr;
   if (b != 0u) {
     const unsigned long long fl = (unsigned long long)b << (32 + kHShift);
@@ -132,6 +132,181 @@ __device__ __forceinline__ int fused_compact_at(int cap, int K) {
   return HIST ? guard : min(guard, max(4 * K, 1024));
 }
 
+// Where a single-token row's selection goes: the output row, and the
+// candidate slots, threshold and arrival counter used when the row is split
+// into segments over several CTAs.
+struct RowOut {
+  int32_t* idx_out;  // [rows][K]
+  float* val_out;    // [rows][K] or null
+  int K;
+  uint32_t* cand_bits;
+  int32_t* cand_idx;
+  int64_t slot_stride;
+  unsigned long long* row_thr;  // per row, zero between calls
+  int32_t* arrive;              // per row, zero between calls
+};
+
+// Segment end of single-token row b in chunk j, the row spanning chunks
+// j0..j1 (all select threads, after a barrier that completed every offer).
+// The filter's digit histogram is exact for its buffer: one warp reads from
+// it the digit b0 of the segment's K-th largest entry, so every entry of the
+// segment's top K is >= vlo = b0's floor.  A segment that holds its whole row
+// takes the exact ordered top K above vlo from registers (fine select,
+// fsel.cuh).  Otherwise it publishes every entry >= vlo, unordered (about K
+// plus one digit bin's worth), raises the row's threshold to vlo, and the
+// last segment to arrive runs the fine select over all published entries.
+static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, int j, int j0,
+                                     int j1) {
+  SelectScratch& sc = *f.sc;
+  FilterState& fs = f.fst[0];
+  uint32_t* fb = f.fbuf;
+  uint32_t* fi = f.fbuf + f.cap;
+  const bool single = j0 == j1;
+  const int nslots = j1 - j0 + 1;
+  int32_t* out_i = o.idx_out + (int64_t)b * o.K;
+  float* out_v = o.val_out ? o.val_out + (int64_t)b * o.K : nullptr;
+  const int64_t slot = (int64_t)(j + b);
+  uint32_t* cbits = o.cand_bits + slot * o.slot_stride;
+  int32_t* cidx = o.cand_idx + slot * o.slot_stride;
+  unsigned long long* row_thr = o.row_thr + b;
+  // Entries per published list: as many as the merge can hold in registers
+  // (kFilterCap over all lists), at least K, at most a slot, a multiple of 4
+  // (lists are copied 16 bytes at a time).
+  const int lcap = max((o.K + 3) & ~3, min((int)o.slot_stride, kFilterCap / nslots) & ~3);
+  // The areas: the fine histogram and its bin offsets in the second radix
+  // histogram of the scratch, the winners in the sort staging, the boundary
+  // list at the front of the buffer once the buffer is in registers.
+  uint32_t* fine = &sc.hist[1][0];
+  const FineArea ar{fine,    fine + kFineBins, f.sortv, f.sortb,
+                    reinterpret_cast<uint64_t*>(f.fbuf), f.fbuf + 2 * (kFineBoundaryMax + 2),
+                    sc.wsum, sc.bcast};
+  constexpr int E = kFilterCap / kSelThreads;
+  uint64_t v[E];
+  uint32_t bits[E];
+  auto out_emit = [&](int pos, uint64_t x, uint32_t xb) {
+    out_i[pos] = (int32_t)~(uint32_t)x;
+    if (out_v) out_v[pos] = __uint_as_float(xb);
+  };
+  auto out_pad = [&](int pos) {
+    out_i[pos] = -1;
+    if (out_v) out_v[pos] = __uint_as_float(kNegInfBits);
+  };
+  // Every asynchronous poll of the request's threshold has landed (the
+  // next segment may belong to another request).
+  cp_async_wait_all();
+  if ((threadIdx.x >> 5) == 0)
+    warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)o.K, single ? 0u : *f.s_row >> kHShift,
+                     sc.bcast);
+  if (threadIdx.x == 0) {
+    sc.ctr = 0;
+    if (single) *row_thr = 0ull;  // raised while streaming, read by nobody else
+  }
+  if (single) fine_clear<kSelThreads>(ar);
+  const int nk = load_buffer<kSelThreads, E>(fb, fi, fs.count, v, bits);
+  IDX_TRACE(19);
+  group_sync(kSelThreads);
+  // b0: the digit of the segment's K-th largest; bp >= b0: the publish
+  // floor, raised to the request's threshold; n0: entries at or above bp.
+  const uint32_t b0 = sc.bcast[0], bmax = sc.bcast[1], n0 = sc.bcast[2], bp = sc.bcast[3];
+  const uint64_t vlo = (uint64_t)b0 << (32 + kHShift);
+  const uint64_t vpub = (uint64_t)bp << (32 + kHShift);
+  IDX_TRACE(13);
+  bool ok = true;
+  if (single) {
+    const uint32_t khi =
+        bmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((bmax + 1) << kHShift) - 1u;
+    ok = fine_select<kSelThreads, E>(v, bits, nk, vlo, khi, o.K, ar, out_emit, out_pad);
+  } else if (n0 <= (uint32_t)lcap) {
+#pragma unroll
+    for (int k = 0; k < E; ++k)
+      if (k < nk && v[k] >= vpub && v[k] != 0) {
+        const int p = atomicAdd(&sc.ctr, 1);
+        cbits[p] = bits[k];
+        cidx[p] = (int32_t)~(uint32_t)v[k];
+      }
+    for (int p = (int)n0 + (int)threadIdx.x; p < lcap; p += kSelThreads) {
+      cbits[p] = kNegInfBits;
+      cidx[p] = -1;
+    }
+    // with b0 > 0 the segment holds K entries >= vlo: so does its row
+    if (threadIdx.x == 0 && b0 != 0) atomicMax(row_thr, (unsigned long long)vlo);
+  } else {
+    ok = false;
+  }
+  if (!ok) {
+    // a crowded digit bin (heavy ties): exact radix compaction first
+    group_sync(kSelThreads);
+    filter_compact<kSelThreads>(fs, fb, fi, o.K, sc);
+    if (single) {
+      sort_and_write<kSelThreads>(fb, fi, fs.count, o.K, f.sortv, f.sortb, out_i, out_v);
+    } else {
+      publish_candidates<kSelThreads>(fb, fi, fs.count, o.K, fs.thr, cbits, cidx, row_thr);
+      for (int p = o.K + (int)threadIdx.x; p < lcap; p += kSelThreads) {
+        cbits[p] = kNegInfBits;
+        cidx[p] = -1;
+      }
+    }
+  }
+  IDX_TRACE(14);
+  if (!single && arrive_last<kSelThreads>(o.arrive + b, nslots, f.s_flag)) {
+    IDX_TRACE(15);
+    auto slot_of = [=](int i) { return (int64_t)(j0 + i + b); };
+    bool done = false;
+    if (nslots * lcap <= kFilterCap) {
+      // the buffer (already published) receives every list
+      stage_lists<kSelThreads>(nslots, slot_of, o.cand_bits, o.cand_idx, o.slot_stride, lcap,
+                               fb, fi);
+      IDX_TRACE(25);
+      const int nkm = load_buffer<kSelThreads, E>(fb, fi, nslots * lcap, v, bits);
+      uint32_t km = 0;
+#pragma unroll
+      for (int k = 0; k < E; ++k) km = max(km, (uint32_t)(v[k] >> 32));
+      km = __reduce_max_sync(0xFFFFFFFFu, km);
+      if (lane_id() == 0) sc.wsum[threadIdx.x >> 5] = km;
+      if (threadIdx.x == 0) {
+        *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = __ldcg(row_thr);
+        *row_thr = 0ull;  // zero for the next call
+      }
+      fine_clear<kSelThreads>(ar);
+      group_sync(kSelThreads);
+      IDX_TRACE(26);
+      const uint64_t thr = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
+      km = 0;
+#pragma unroll
+      for (int w = 0; w < kSelThreads / 32; ++w) km = max(km, sc.wsum[w]);
+      done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, o.K, ar, out_emit, out_pad);
+      if (!done) {
+        // a crowded boundary bin (heavy ties): the entries at or above the
+        // threshold go back to the buffer for the exact radix compaction
+        if (threadIdx.x == 0) sc.ctr = 0;
+        group_sync(kSelThreads);
+#pragma unroll
+        for (int k = 0; k < E; ++k)
+          if (k < nkm && v[k] >= thr && v[k] != 0) {
+            const int p = atomicAdd(&sc.ctr, 1);
+            fb[p] = bits[k];
+            fi[p] = ~(uint32_t)v[k];
+          }
+        group_sync(kSelThreads);
+        if (threadIdx.x == 0) {
+          fs.count = sc.ctr;
+          fs.thr = 0ull;
+        }
+        group_sync(kSelThreads);
+        filter_compact<kSelThreads>(fs, fb, fi, o.K, sc);
+        sort_and_write<kSelThreads>(fb, fi, fs.count, o.K, f.sortv, f.sortb, out_i, out_v);
+        done = true;
+      }
+    }
+    if (!done)
+      merge_candidates<kSelThreads>(nslots, slot_of, o.cand_bits, o.cand_idx, o.slot_stride,
+                                    lcap, o.K, row_thr, fs, f.fbuf, f.fbuf + kFilterCap,
+                                    kFilterCap, sc, f.sortv, f.sortb, out_i, out_v);
+    IDX_TRACE(16);
+  }
+  group_sync(kSelThreads);
+}
+
 // Segment end for request b, chunk j (all select threads, after a barrier
 // that completed every offer).  The request's pages span chunks j0..j1.
 template <bool HIST>
@@ -139,160 +314,10 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
                                int j1) {
   SelectScratch& sc = *f.sc;
   if (HIST) {
-    // One token per row.  The filter's digit histogram is exact for its
-    // buffer: one warp reads from it the digit b0 of the segment's K-th
-    // largest entry, so every entry of the segment's top K is >= vlo = b0's
-    // floor.  A segment that holds its whole request takes the exact ordered
-    // top K above vlo from registers (fine select, fsel.cuh).  Otherwise it
-    // publishes every entry >= vlo, unordered (about K plus one digit bin's
-    // worth), raises the request's threshold to vlo, and the last segment to
-    // arrive runs the fine select over all published entries.
-    FilterState& fs = f.fst[0];
-    uint32_t* fb = f.fbuf;
-    uint32_t* fi = f.fbuf + f.cap;
-    const bool single = j0 == j1;
-    const int nslots = j1 - j0 + 1;
-    int32_t* out_i = a.idx_out + (int64_t)b * a.K;
-    float* out_v = a.val_out ? a.val_out + (int64_t)b * a.K : nullptr;
-    const int64_t slot = (int64_t)(j + b);
-    uint32_t* cbits = a.cand_bits + slot * a.slot_stride;
-    int32_t* cidx = a.cand_idx + slot * a.slot_stride;
-    unsigned long long* row_thr = a.row_thr + b;
-    // Entries per published list: as many as the merge can hold in registers
-    // (kFilterCap over all lists), at least K, at most a slot, a multiple of 4
-    // (lists are copied 16 bytes at a time).
-    const int lcap = max((a.K + 3) & ~3, min((int)a.slot_stride, kFilterCap / nslots) & ~3);
-    // The areas: the fine histogram and its bin offsets in the second radix
-    // histogram of the scratch, the winners in the sort staging, the boundary
-    // list at the front of the buffer once the buffer is in registers.
-    uint32_t* fine = &sc.hist[1][0];
-    const FineArea ar{fine,    fine + kFineBins, f.sortv, f.sortb,
-                      reinterpret_cast<uint64_t*>(f.fbuf), f.fbuf + 2 * (kFineBoundaryMax + 2),
-                      sc.wsum, sc.bcast};
-    constexpr int E = kFilterCap / kSelThreads;
-    uint64_t v[E];
-    uint32_t bits[E];
-    auto out_emit = [&](int pos, uint64_t x, uint32_t xb) {
-      out_i[pos] = (int32_t)~(uint32_t)x;
-      if (out_v) out_v[pos] = __uint_as_float(xb);
-    };
-    auto out_pad = [&](int pos) {
-      out_i[pos] = -1;
-      if (out_v) out_v[pos] = __uint_as_float(kNegInfBits);
-    };
-    // Every asynchronous poll of the request's threshold has landed (the
-    // next segment may belong to another request).
-    cp_async_wait_all();
-    if ((threadIdx.x >> 5) == 0)
-      warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)a.K, single ? 0u : *f.s_row >> kHShift,
-                       sc.bcast);
-    if (threadIdx.x == 0) {
-      sc.ctr = 0;
-      if (single) *row_thr = 0ull;  // raised while streaming, read by nobody else
-    }
-    if (single) fine_clear<kSelThreads>(ar);
-    const int nk = load_buffer<kSelThreads, E>(fb, fi, fs.count, v, bits);
-    IDX_TRACE(19);
-    group_sync(kSelThreads);
-    // b0: the digit of the segment's K-th largest; bp >= b0: the publish
-    // floor, raised to the request's threshold; n0: entries at or above bp.
-    const uint32_t b0 = sc.bcast[0], bmax = sc.bcast[1], n0 = sc.bcast[2], bp = sc.bcast[3];
-    const uint64_t vlo = (uint64_t)b0 << (32 + kHShift);
-    const uint64_t vpub = (uint64_t)bp << (32 + kHShift);
-    IDX_TRACE(13);
-    bool ok = true;
-    if (single) {
-      const uint32_t khi =
-          bmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((bmax + 1) << kHShift) - 1u;
-      ok = fine_select<kSelThreads, E>(v, bits, nk, vlo, khi, a.K, ar, out_emit, out_pad);
-    } else if (n0 <= (uint32_t)lcap) {
-#pragma unroll
-      for (int k = 0; k < E; ++k)
-        if (k < nk && v[k] >= vpub && v[k] != 0) {
-          const int p = atomicAdd(&sc.ctr, 1);
-          cbits[p] = bits[k];
-          cidx[p] = (int32_t)~(uint32_t)v[k];
-        }
-      for (int p = (int)n0 + (int)threadIdx.x; p < lcap; p += kSelThreads) {
-        cbits[p] = kNegInfBits;
-        cidx[p] = -1;
-      }
-      // with b0 > 0 the segment holds K entries >= vlo: so does its row
-      if (threadIdx.x == 0 && b0 != 0) atomicMax(row_thr, (unsigned long long)vlo);
-    } else {
-      ok = false;
-    }
-    if (!ok) {
-      // a crowded digit bin (heavy ties): exact radix compaction first
-      group_sync(kSelThreads);
-      filter_compact<kSelThreads>(fs, fb, fi, a.K, sc);
-      if (single) {
-        sort_and_write<kSelThreads>(fb, fi, fs.count, a.K, f.sortv, f.sortb, out_i, out_v);
-      } else {
-        publish_candidates<kSelThreads>(fb, fi, fs.count, a.K, fs.thr, cbits, cidx, row_thr);
-        for (int p = a.K + (int)threadIdx.x; p < lcap; p += kSelThreads) {
-          cbits[p] = kNegInfBits;
-          cidx[p] = -1;
-        }
-      }
-    }
-    IDX_TRACE(14);
-    if (!single && arrive_last<kSelThreads>(a.arrive + b, nslots, f.s_flag)) {
-      IDX_TRACE(15);
-      auto slot_of = [=](int i) { return (int64_t)(j0 + i + b); };
-      bool done = false;
-      if (nslots * lcap <= kFilterCap) {
-        // the buffer (already published) receives every list
-        stage_lists<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride, lcap,
-                                 fb, fi);
-        IDX_TRACE(25);
-        const int nkm = load_buffer<kSelThreads, E>(fb, fi, nslots * lcap, v, bits);
-        uint32_t km = 0;
-#pragma unroll
-        for (int k = 0; k < E; ++k) km = max(km, (uint32_t)(v[k] >> 32));
-        km = __reduce_max_sync(0xFFFFFFFFu, km);
-        if (lane_id() == 0) sc.wsum[threadIdx.x >> 5] = km;
-        if (threadIdx.x == 0) {
-          *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = __ldcg(row_thr);
-          *row_thr = 0ull;  // zero for the next call
-        }
-        fine_clear<kSelThreads>(ar);
-        group_sync(kSelThreads);
-        IDX_TRACE(26);
-        const uint64_t thr = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
-        km = 0;
-#pragma unroll
-        for (int w = 0; w < kSelThreads / 32; ++w) km = max(km, sc.wsum[w]);
-        done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, a.K, ar, out_emit, out_pad);
-        if (!done) {
-          // a crowded boundary bin (heavy ties): the entries at or above the
-          // threshold go back to the buffer for the exact radix compaction
-          if (threadIdx.x == 0) sc.ctr = 0;
-          group_sync(kSelThreads);
-#pragma unroll
-          for (int k = 0; k < E; ++k)
-            if (k < nkm && v[k] >= thr && v[k] != 0) {
-              const int p = atomicAdd(&sc.ctr, 1);
-              fb[p] = bits[k];
-              fi[p] = ~(uint32_t)v[k];
-            }
-          group_sync(kSelThreads);
-          if (threadIdx.x == 0) {
-            fs.count = sc.ctr;
-            fs.thr = 0ull;
-          }
-          group_sync(kSelThreads);
-          filter_compact<kSelThreads>(fs, fb, fi, a.K, sc);
-          sort_and_write<kSelThreads>(fb, fi, fs.count, a.K, f.sortv, f.sortb, out_i, out_v);
-          done = true;
-        }
-      }
-      if (!done)
-        merge_candidates<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride,
-                                      lcap, a.K, row_thr, fs, f.fbuf, f.fbuf + kFilterCap,
-                                      kFilterCap, sc, f.sortv, f.sortb, out_i, out_v);
-      IDX_TRACE(16);
-    }
+    const RowOut o{a.idx_out,     a.val_out, a.K,       a.cand_bits,
+                   a.cand_idx,    a.slot_stride, a.row_thr, a.arrive};
+    hist_finalize(f, o, b, j, j0, j1);
+    return;
   } else {
     for (int t = 0; t < T; ++t) {
       uint32_t* fb = f.fbuf + t * 2 * f.cap;

@@ -110,6 +110,41 @@ __device__ __forceinline__ uint32_t hist_floor_1t(const uint32_t* hist, const ui
   return 0u;
 }
 
+// hist_floor_1t computed by a whole warp (every lane gets the result): lane l
+// reads the 4 coarse bins 4(31 - l) .. 4(31 - l) + 3 (lane 0 the top ones),
+// one inclusive scan finds the coarse bin that reaches K, and one more over
+// its 32 fine bins the digit.  About a dozen dependent steps instead of a
+// serial walk down the bins.
+__device__ __forceinline__ uint32_t hist_floor_warp(const uint32_t* hist, const uint32_t* chist,
+                                                    uint32_t K) {
+  const uint32_t lane = lane_id();
+  const uint4 q = reinterpret_cast<const uint4*>(chist)[31 - lane];
+  const uint32_t ch[4] = {q.w, q.z, q.y, q.x};
+  const uint32_t s4 = q.x + q.y + q.z + q.w;
+  const uint32_t incl = warp_incl_scan(s4);
+  const uint32_t hit = __ballot_sync(0xFFFFFFFFu, incl - s4 < K && incl >= K);
+  if (!hit) return 0u;  // fewer than K entries counted
+  const int l = __ffs(hit) - 1;
+  uint32_t cum = incl - s4, cb = 0, before = 0;
+  bool found = false;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if (!found && cum + ch[e] >= K) {
+      cb = 4 * (31 - lane) + 3 - e;
+      before = cum;
+      found = true;
+    }
+    cum += ch[e];
+  }
+  cb = __shfl_sync(0xFFFFFFFFu, cb, l);
+  before = __shfl_sync(0xFFFFFFFFu, before, l);
+  const uint32_t fi = warp_incl_scan(hist[32 * cb + 31 - lane]) + before;
+  const uint32_t fh = __ballot_sync(0xFFFFFFFFu, fi >= K);
+  // counts only grow while the warp reads them: a racy read may find K only
+  // in the coarse count, and bin 32 cb is then still a valid floor
+  return fh ? 32 * cb + 31 - (uint32_t)(__ffs(fh) - 1) : 32 * cb;
+}
+
 // Raise a filter's threshold to "digit >= b" (one thread).  A racing raise by
 // another warp may win with a lower value: that only admits more entries.
 __device__ __forceinline__ void raise_threshold_1t(FilterState& fs, const uint32_t* hist,

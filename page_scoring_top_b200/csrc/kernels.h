@@ -31,6 +31,32 @@ struct TopkArgs {
 int topk_plan_chunk(int rows, int N, int K, int num_sms);
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 
+// Streamed top-K (topk_stream.cu): one persistent CTA per SM over the rows laid
+// end to end.  Needs 16-byte aligned scores and lds % 4 == 0; at most
+// topk_stream_max_rows() rows per launch; candidate slots (chunk + row) of
+// slot_stride entries, and per-row thresholds and arrival counters that are
+// zero between calls.
+struct TopkStreamArgs {
+  const float* scores;
+  const int32_t* lengths;  // or null (all N); row r uses lengths[r / len_div]
+  int len_div;
+  int rows, N;
+  int64_t lds;
+  int K;
+  int32_t* idx_out;
+  float* val_out;  // may be null
+  uint32_t* cand_bits;
+  int32_t* cand_idx;
+  int64_t slot_stride;
+  unsigned long long* row_thr;
+  int32_t* arrive;
+  int* status;
+};
+bool topk_stream_supported(const float* scores, int64_t lds);
+int64_t topk_stream_slots(int rows, int num_sms);
+int topk_stream_max_rows();
+cudaError_t launch_topk_stream(const TopkStreamArgs& a, int num_sms, cudaStream_t stream);
+
 // ---------------------------------------------------------------- decode score / fused select
 struct DecodeArgs {
   const uint16_t* q;
