@@ -57,12 +57,15 @@ def _load():
         lib.oracle_scores.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
         lib.oracle_scores_tokens.argtypes = [P, P, P, I, I, I, I, I, L, P, P]
         lib.oracle_pool.argtypes = [P, P, I, I, I, I, L, P]
+        lib.oracle_kmeans_assign.argtypes = [P, P, I, I, I, P, P, P, P]
+        lib.oracle_argmax_rows_f32.argtypes = [P, I, I, P]
         lib.oracle_topk_f64.argtypes = [P, I, I, P, P]
         lib.oracle_topk_f32.argtypes = [P, I, I, P, P]
         lib.oracle_topk_rows_f32.argtypes = [P, P, I, I, L, I, P, P]
         lib.oracle_topk_rows_f64.argtypes = [P, P, I, I, L, I, P, P]
         for f in ("oracle_scores", "oracle_scores_tokens", "oracle_pool", "oracle_topk_f64",
-                  "oracle_topk_f32", "oracle_topk_rows_f32", "oracle_topk_rows_f64"):
+                  "oracle_topk_f32", "oracle_topk_rows_f32", "oracle_topk_rows_f64",
+                  "oracle_kmeans_assign", "oracle_argmax_rows_f32"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -136,6 +139,40 @@ def scores_paged(q_bits, pool_bits, page_table, lengths=None):
     gathered = pool[np.where(live, pt, 0)]  # [B][N][D]; dead pages read block 0, then masked
     gathered = np.where(live[:, :, None], gathered, np.uint16(0))
     return scores(q_bits, gathered, lengths)
+
+
+def kmeans_assign(x_bits, c_bits, full=False):
+    """Nearest centroid of every point (the KMeans assignment of "Export Cake
+    KMeans plan-runtime suite"): argmax_c (x.c - |c|^2/2) in double, ties to
+    the lower centroid.  ``x_bits`` uint16 bf16 [M][D], ``c_bits`` [C][D].
+    Returns (assign int32 [M], best double [M]) and, with ``full``, also the
+    score matrix S and its error-bound scale A, double [M][C]."""
+    x = _c(x_bits, np.uint16)
+    c = _c(c_bits, np.uint16)
+    M, D = x.shape
+    C, Dc = c.shape
+    assert Dc == D
+    assign = np.empty(M, np.int32)
+    best = np.empty(M, np.float64)
+    S = np.empty((M, C), np.float64) if full else None
+    A = np.empty((M, C), np.float64) if full else None
+    rc = _load().oracle_kmeans_assign(_ptr(x), _ptr(c), M, C, D, _ptr(assign), _ptr(best),
+                                      _ptr(S), _ptr(A))
+    if rc != 0:
+        raise ValueError("oracle_kmeans_assign: arguments outside the contract")
+    return (assign, best, S, A) if full else (assign, best)
+
+
+def argmax_rows(scores_f32):
+    """Column of the largest entry of every row of an fp32 matrix (ties to the
+    lower column, NaN never wins)."""
+    s = _c(scores_f32, np.float32)
+    M, C = s.shape
+    arg = np.empty(M, np.int32)
+    rc = _load().oracle_argmax_rows_f32(_ptr(s), M, C, _ptr(arg))
+    if rc != 0:
+        raise ValueError("oracle_argmax_rows_f32: arguments outside the contract")
+    return arg
 
 
 def topk(row, K, length=None):

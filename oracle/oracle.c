@@ -274,3 +274,73 @@ ORACLE_API int oracle_pool(const uint16_t* keys, const int32_t* key_counts, int 
     }
     return 0;
 }
+
+/*
+ * KMeans assignment ("Export Cake KMeans plan-runtime suite", summary:
+ * assignments = runtime.compute(x, centroids) on raw bf16 inputs): every
+ * point goes to its nearest centroid in Euclidean distance.  Since
+ * |x - c|^2 = |x|^2 - 2 (x.c - |c|^2 / 2) and |x|^2 does not depend on c,
+ * the nearest centroid is the one of largest
+ *     s[i,c] = sum_d x[i,d] * c[c,d] - (sum_d c[c,d]^2) / 2,
+ * computed here in double (bf16 products and squares are exact in double).
+ * Equal scores go to the lower centroid index.
+ *   x       bf16 bits [M][D], centroids bf16 bits [C][D]
+ *   assign  int32 [M]; best double [M] (the winning score)
+ *   S, A    optional (NULL) double [M][C]: every score, and the scale of its
+ *           error bound, sum_d |x*c| + (sum_d c^2) / 2
+ * Returns -1 on arguments outside the contract.
+ */
+ORACLE_API int oracle_kmeans_assign(const uint16_t* x, const uint16_t* cent, int M, int C, int D,
+                                    int32_t* assign, double* best, double* S, double* A)
+{
+    if (M < 0 || C <= 0 || D <= 0 || !assign || !best) return -1;
+    for (int i = 0; i < M; ++i) {
+        int arg = 0;
+        double top = 0.0;
+        for (int c = 0; c < C; ++c) {
+            double dot = 0.0, mag = 0.0, half = 0.0;
+            for (int d = 0; d < D; ++d) {
+                const double xv = bf16_bits_to_double(x[(int64_t)i * D + d]);
+                const double cv = bf16_bits_to_double(cent[(int64_t)c * D + d]);
+                dot += xv * cv;
+                mag += fabs(xv * cv);
+                half += cv * cv;
+            }
+            half *= 0.5;
+            const double s = dot - half;
+            if (S) S[(int64_t)i * C + c] = s;
+            if (A) A[(int64_t)i * C + c] = mag + half;
+            if (c == 0 || s > top) {  /* strictly greater: ties keep the lower index */
+                top = s;
+                arg = c;
+            }
+        }
+        assign[i] = arg;
+        best[i] = top;
+    }
+    return 0;
+}
+
+/*
+ * Argmax of every row of an fp32 score matrix [M][C] (ties to the lower
+ * column; NaN never wins, a row of NaN gives -1), for the bit-exact check of
+ * an assignment against the GPU's own scores.
+ */
+ORACLE_API int oracle_argmax_rows_f32(const float* S, int M, int C, int32_t* arg)
+{
+    if (M < 0 || C <= 0 || !arg) return -1;
+    for (int i = 0; i < M; ++i) {
+        int a = -1;
+        float top = 0.0f;
+        for (int c = 0; c < C; ++c) {
+            const float v = S[(int64_t)i * C + c];
+            if (v != v) continue;
+            if (a < 0 || v > top) {
+                top = v;
+                a = c;
+            }
+        }
+        arg[i] = a;
+    }
+    return 0;
+}

@@ -470,3 +470,78 @@ def test_paged_scores_reject_ids_outside_the_pool():
         oracle.scores_paged(q, pool, np.array([[-1, 0]], np.int32), np.array([2], np.int32))
     S, _ = oracle.scores_paged(q, pool, np.array([[1, 99]], np.int32), np.array([1], np.int32))
     assert S[0, 0].tolist() == [2.0, -np.inf]
+
+
+# ------------------------------------------------------------------ KMeans assignment
+# "Export Cake KMeans plan-runtime suite" (summary): assignments =
+# compute(x, centroids), each point to its nearest centroid.
+
+def test_kmeans_worked_example():
+    # centroids (0,0), (2,0), (0,2); by hand:
+    #   (1.5, 0.25): squared distances 2.3125, 0.3125, 5.3125 -> centroid 1,
+    #                score x.c - |c|^2/2 = 3 - 2 = 1
+    #   (0.25, 0.25): 0.125, 3.125, 3.125 -> centroid 0, score 0
+    #   (1, 1): 2, 2, 2 -> a three-way tie, the lowest index 0, score 0
+    x = _bf16([[1.5, 0.25], [0.25, 0.25], [1.0, 1.0]])
+    c = _bf16([[0.0, 0.0], [2.0, 0.0], [0.0, 2.0]])
+    assign, best = oracle.kmeans_assign(x, c)
+    assert assign.tolist() == [1, 0, 0]
+    assert best.tolist() == [1.0, 0.0, 0.0]
+
+
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_kmeans_matches_nearest_by_distance(seed):
+    # an independent formulation: argmin of the squared Euclidean distance,
+    # library arithmetic in double (exact for these bf16 inputs), first minimum
+    rng = np.random.default_rng(seed)
+    M, C, D = 37, 11, 16
+    xf = rng.integers(-8, 9, size=(M, D)).astype(np.float32) / 4
+    cf = rng.integers(-8, 9, size=(C, D)).astype(np.float32) / 4
+    x, c = synth.f32_to_bf16_bits(xf), synth.f32_to_bf16_bits(cf)
+    assign, best, S, A = oracle.kmeans_assign(x, c, full=True)
+    d2 = ((xf.astype(np.float64)[:, None, :] - cf.astype(np.float64)[None, :, :]) ** 2).sum(-1)
+    assert np.array_equal(assign, np.argmin(d2, axis=1))
+    # the score is the library's x c^T - |c|^2 / 2, and the winner's score is best
+    lib = xf.astype(np.float64) @ cf.astype(np.float64).T - 0.5 * (cf.astype(np.float64) ** 2).sum(1)
+    assert np.array_equal(S, lib)
+    assert np.array_equal(best, S[np.arange(M), assign])
+    assert np.all(A >= np.abs(S))
+
+
+def test_kmeans_invariants():
+    rng = np.random.default_rng(7)
+    M, C, D = 50, 9, 8
+    cf = rng.standard_normal((C, D)).astype(np.float32)
+    c = synth.f32_to_bf16_bits(cf)
+    # a point on a centroid goes to it (distinct centroids)
+    x = c[[4, 0, 8]]
+    assert oracle.kmeans_assign(x, c)[0].tolist() == [4, 0, 8]
+    # permuting the centroids permutes the assignment (no ties at random)
+    x = synth.f32_to_bf16_bits(rng.standard_normal((M, D)).astype(np.float32))
+    a0, _ = oracle.kmeans_assign(x, c)
+    perm = rng.permutation(C)
+    a1, _ = oracle.kmeans_assign(x, c[perm])
+    assert np.array_equal(perm[a1], a0)
+    # doubling x (exact in bf16) and centroids leaves the nearest centroid
+    x2 = synth.f32_to_bf16_bits(2 * synth.bf16_bits_to_f32(x))
+    c2 = synth.f32_to_bf16_bits(2 * synth.bf16_bits_to_f32(c))
+    assert np.array_equal(oracle.kmeans_assign(x2, c2)[0], a0)
+
+
+def test_argmax_rows_ties_and_nan():
+    s = np.array([[1.0, 3.0, 3.0, 2.0], [np.nan, -1.0, np.nan, -1.0],
+                  [np.nan, np.nan, np.nan, np.nan], [-0.0, 0.0, 0.0, -5.0]], np.float32)
+    assert oracle.argmax_rows(s).tolist() == [1, 1, -1, 0]
+
+
+def test_kmeans_checker_rejects_planted_mistakes():
+    # a plausible wrong rule (no half on |c|^2, or + instead of -) changes
+    # the assignment on this example
+    x = _bf16([[1.5, 0.25], [0.25, 0.25]])
+    c = _bf16([[0.0, 0.0], [2.0, 0.0]])
+    xf, cf = synth.bf16_bits_to_f32(x).astype(np.float64), synth.bf16_bits_to_f32(c).astype(np.float64)
+    good = oracle.kmeans_assign(x, c)[0]
+    no_half = np.argmax(xf @ cf.T - (cf ** 2).sum(1), axis=1)
+    plus = np.argmax(xf @ cf.T + 0.5 * (cf ** 2).sum(1), axis=1)
+    assert good.tolist() == [1, 0]
+    assert no_half.tolist() != good.tolist() and plus.tolist() != good.tolist()
