@@ -67,7 +67,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=("ragged_decode", "prefill_chunk", "causal_decode", "pool_keys",
-                             "paged_decode", "topk_sweep",
+                             "paged_decode", "topk_sweep", "kmeans_assign",
                              "batch_decode_bias", "tiny_decode"))
     ap.add_argument("--dists", default="normal,levels16,neg_inf_90",
                     help="top-K sweep distributions (comma list, or 'all')")
@@ -177,6 +177,16 @@ def measured_peak():
             return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s: the measured burst figure, else the recipe's fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        return 1590.0, "fallback (1.59 PFLOP/s earlier pool measurement, burst)"
 
 
 class ClockSampler:
@@ -713,6 +723,62 @@ def run_topk_sweep(args):
     return 0
 
 
+def run_kmeans(args):
+    """KMeans assignment, the second workload: 262144 clustered points, 1024
+    centroids, D=128 (seed 109), one kmeans_assign call per step (the h
+    pre-pass and the tcgen05 assignment kernel).  Units are points assigned;
+    the roofline is the tensor pipe (2 M C D flops per step)."""
+    import torch
+    from page_scoring_top_b200 import binding, synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    spec = synth.KMEANS
+    M, C, D = spec["M"], spec["C"], spec["D"]
+    d = synth.kmeans_inputs(spec["seed"], M, C, D)
+    xd = torch.from_numpy(d["x"].view(np.int16)).to(dev)
+    cd = torch.from_numpy(d["centroids"].view(np.int16)).to(dev)
+    assign = torch.empty(M, dtype=torch.int32, device=dev)
+    ctx = binding.Context(0, max_rows=1, max_n=C, max_k=1)
+    stream = torch.cuda.current_stream(dev)
+    step = lambda: binding.kmeans_assign(ctx, xd, cd, assign, None, stream=stream)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.15)
+    soak(step, 0.3)
+    reps = timed_repeats(step, args.steps, stream, lambda: None)
+    clocks = sampler.stop()
+    ms = float(np.median(reps)) / args.steps
+    rc, bits = binding.idx_get_status(ctx)
+    if rc != 0:
+        raise RuntimeError("device status %d" % bits)
+    flops = 2.0 * M * C * D
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak, peak_src = measured_tensor_peak()
+    nbytes = M * D * 2 + C * D * 2 + M * 4
+    line = {
+        "metric": "points assigned/sec (KMeans assignment, nearest of 1024 centroids)",
+        "value": M / (ms * 1e-3), "unit": "points/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "accumulate": "f32", "data": "synthetic",
+        "config": {"workload": "kmeans_assign", "M": M, "C": C, "D": D, "seed": spec["seed"],
+                   "points": "clustered: a uniform centroid + 0.5 N(0,1)",
+                   "l2": "inputs (%.0f MB of points) larger than half the L2, back to back"
+                         % (M * D * 2 / 1e6)},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None, "peak_source": peak_src,
+                     "kernel": "kmeans_kernel (tcgen05 M128 N256, argmax epilogue)",
+                     "hbm_gbs": nbytes / (ms * 1e-3) / 1e9},
+        "repeats": {"regions": len(reps), "ms_per_step": [r / args.steps for r in reps]},
+        "gpu_launches": 2 * args.steps, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    ctx.close()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -723,6 +789,8 @@ def main():
         return run_paged(args)
     if args.workload == "topk_sweep":
         return run_topk_sweep(args)
+    if args.workload == "kmeans_assign":
+        return run_kmeans(args)
     return run_ours(args)
 
 

@@ -179,6 +179,30 @@ IDX_API int centroid_pool(idx_ctx* ctx, const uint16_t* keys, const int32_t* key
                           idx_stream stream);
 
 /*
+ * KMeans assignment, the second workload of the library ("Export Cake KMeans
+ * plan-runtime suite", summary: assignments = compute(x, centroids) on raw
+ * bf16 inputs): every point goes to its nearest centroid in Euclidean
+ * distance, i.e. to
+ *     assign[i] = argmax_c s[i,c],  s[i,c] = sum_d x[i,d] * c[c,d] - h[c],
+ *     h[c] = (sum_d c[c,d]^2) / 2,
+ * equal scores to the lower centroid index.  x: bf16 [M][D], centroids: bf16
+ * [C][D], both contiguous and 16-byte aligned; D a multiple of 8, at most 128.
+ * The dot products run on the tensor cores (tcgen05, fp32 accumulation in
+ * TMEM), h in fp32; every s is within 1e-5 * (sum_d |x*c| + h) of the exact
+ * score.  The two-stage shape of that page (init() once, compute() many
+ * times) is idx_init then these calls.  h lives in the context's score
+ * workspace: C <= max_rows * max_n of idx_init, else IDX_ENOWORKSPACE.
+ * kmeans_assign writes assign_out int32 [M] and, if score_out is non-NULL,
+ * the winning score fp32 [M].  kmeans_scores writes every s, fp32 [M][C]
+ * (16-byte aligned), from the same arithmetic: kmeans_assign's output is the
+ * row argmax of kmeans_scores' output, bit for bit.
+ */
+IDX_API int kmeans_assign(idx_ctx* ctx, const uint16_t* x, const uint16_t* centroids, int M, int C,
+                          int D, int32_t* assign_out, float* score_out, idx_stream stream);
+IDX_API int kmeans_scores(idx_ctx* ctx, const uint16_t* x, const uint16_t* centroids, int M, int C,
+                          int D, float* scores, idx_stream stream);
+
+/*
  * Device-side status of the context: waits for `stream`, reads and clears the
  * status word.  Returns IDX_OK, or IDX_EDEVICE with *bits (if non-NULL) set to
  * the raised bits: 1 = a length outside [0, N] was clamped, 2 = a bounded wait

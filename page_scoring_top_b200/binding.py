@@ -42,6 +42,8 @@ SIGNATURES = {
     "idx_strerror": (ctypes.c_char_p, [_I]),
     "idx_num_sms": (_I, [_P]),
     "topk_select_noalloc": (_I, [_P, _P, _I, _I, _L, _I, _P, _P, _P]),
+    "kmeans_assign": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
+    "kmeans_scores": (_I, [_P, _P, _P, _I, _I, _I, _P, _P]),
 }
 
 _lib = None
@@ -242,6 +244,36 @@ def centroid_pool(ctx, keys, key_counts, P, c, stream=None):
     _check(lib().centroid_pool(ctx.handle, _ptr(keys), _ptr(key_counts), B, D, P, N, Lk * D,
                                _ptr(c), N * D, _stream(stream, keys.device)), "centroid_pool")
     return c
+
+
+def _kmeans_shapes(x, centroids):
+    for name, t in (("x", x), ("centroids", centroids)):
+        if t.dim() != 2 or t.dtype not in (torch.int16, torch.bfloat16) or not t.is_contiguous():
+            raise ValueError("%s must be contiguous bf16 (or its int16 bits) [rows][D]" % name)
+    M, D = x.shape
+    C, Dc = centroids.shape
+    if Dc != D:
+        raise ValueError("x and centroids differ in D")
+    return M, C, D
+
+
+def kmeans_assign(ctx, x, centroids, assign_out, score_out=None, stream=None):
+    """assign_out[i] = nearest centroid of point i (int32 [M]); score_out, if
+    given, gets the winning x.c - |c|^2/2 (fp32 [M])."""
+    M, C, D = _kmeans_shapes(x, centroids)
+    _check(lib().kmeans_assign(ctx.handle, _ptr(x), _ptr(centroids), M, C, D, _ptr(assign_out),
+                               _ptr(score_out), _stream(stream, x.device)), "kmeans_assign")
+    return assign_out, score_out
+
+
+def kmeans_scores(ctx, x, centroids, scores, stream=None):
+    """scores[i, c] = x_i.c - |c|^2/2 (fp32 [M][C])."""
+    M, C, D = _kmeans_shapes(x, centroids)
+    if tuple(scores.shape) != (M, C) or scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be contiguous fp32 [M][C]")
+    _check(lib().kmeans_scores(ctx.handle, _ptr(x), _ptr(centroids), M, C, D, _ptr(scores),
+                               _stream(stream, x.device)), "kmeans_scores")
+    return scores
 
 
 def _paged_shapes(q, pool, page_table):

@@ -470,6 +470,45 @@ IDX_API int score_topk_fused_tokens(idx_ctx* ctx, const uint16_t* q, const uint1
                     stream);
 }
 
+// KMeans assignment and scores: x [M][D], centroids [C][D] (bf16, 16-byte
+// aligned), h = |c|^2/2 in the context's score scratch (C floats).
+static int kmeans_impl(idx_ctx* ctx, const uint16_t* x, const uint16_t* cent, int M, int C, int D,
+                       int32_t* assign, float* score, float* scores, idx_stream stream) {
+  if (!ctx || !x || !cent) return IDX_EINVAL;
+  if (M <= 0 || C <= 0 || D <= 0) return IDX_EINVAL;
+  if (!aligned16(x) || !aligned16(cent)) return IDX_EINVAL;
+  if ((D % 8) != 0) return IDX_EINVAL;
+  if (!idx::kmeans_supported(D)) return IDX_EUNSUPPORTED;
+  if ((int64_t)C > ctx->scratch_elems) return IDX_ENOWORKSPACE;
+  DeviceGuard guard(ctx->device);
+  if (!guard.ok()) return IDX_ECUDA;
+  idx::KmeansArgs a{};
+  a.x = x;
+  a.cent = cent;
+  a.M = M;
+  a.C = C;
+  a.D = D;
+  a.hn = ctx->scratch;
+  a.assign = assign;
+  a.score = score;
+  a.scores = scores;
+  a.status = ctx->status;
+  return status_of(idx::launch_kmeans(a, scores != nullptr, ctx->num_sms, (cudaStream_t)stream));
+}
+
+IDX_API int kmeans_assign(idx_ctx* ctx, const uint16_t* x, const uint16_t* centroids, int M, int C,
+                          int D, int32_t* assign_out, float* score_out, idx_stream stream) {
+  if (!assign_out) return IDX_EINVAL;
+  return kmeans_impl(ctx, x, centroids, M, C, D, assign_out, score_out, nullptr, stream);
+}
+
+IDX_API int kmeans_scores(idx_ctx* ctx, const uint16_t* x, const uint16_t* centroids, int M, int C,
+                          int D, float* scores, idx_stream stream) {
+  if (!scores || !aligned16(scores)) return IDX_EINVAL;
+  if ((int64_t)M * C > INT32_MAX * 4ll) return IDX_EUNSUPPORTED;
+  return kmeans_impl(ctx, x, centroids, M, C, D, nullptr, nullptr, scores, stream);
+}
+
 IDX_API int idx_get_status(idx_ctx* ctx, idx_stream stream, int* bits) {
   if (!ctx) return IDX_EINVAL;
   DeviceGuard guard(ctx->device);

@@ -108,6 +108,21 @@ constexpr int kPrefillMaxB = 256;  // requests per launch (host splits larger ba
 bool prefill_supported(int T, int Q, int D, int64_t ldc_b);
 cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t stream);
 
+// ---------------------------------------------------------------- KMeans assignment
+struct KmeansArgs {
+  const uint16_t* x;     // bf16 [M][D], 16-byte aligned rows
+  const uint16_t* cent;  // bf16 [C][D]
+  int M, C, D;
+  float* hn;             // [C] workspace: |c|^2 / 2
+  int32_t* assign;       // [M] (assignment mode)
+  float* score;          // [M] or null (assignment mode)
+  float* scores;         // [M][C] (score mode)
+  int* status;
+};
+bool kmeans_supported(int D);
+// Computes hn, then the assignment (scores == false) or the score matrix.
+cudaError_t launch_kmeans(const KmeansArgs& a, bool scores, int num_sms, cudaStream_t stream);
+
 // ---------------------------------------------------------------- page centroids
 struct PoolArgs {
   const uint16_t* keys;        // bf16, key i of request b at keys + b*ldk_b + i*D

@@ -275,3 +275,24 @@ def workload(name, **override):
                            spec.pop("D"), spec.pop("N"), **spec)
     inputs["K"] = K
     return inputs
+
+
+# --------------------------------------------------------------------------
+# KMeans assignment inputs (the second workload)
+# --------------------------------------------------------------------------
+
+KMEANS = dict(seed=109, M=262144, C=1024, D=128)
+
+
+def kmeans_inputs(seed, M, C, D, spread=0.5):
+    """Clustered points for an assignment: centroids ~ N(0,1) (stream 1), each
+    point a centroid chosen uniformly (stream 2) plus ``spread`` * N(0,1)
+    noise (stream 3), rounded once to bf16.  Returns bf16 bits x [M][D],
+    centroids [C][D] and the generating centroid of every point."""
+    cf = normal(seed, 1, 0, C * D).astype(np.float32).reshape(C, D)
+    cent = f32_to_bf16_bits(cf)
+    cf = bf16_bits_to_f32(cent)
+    pick = (u64(seed, 2, 0, M) % np.uint64(C)).astype(np.int64)
+    noise = normal(seed, 3, 0, M * D).astype(np.float32).reshape(M, D)
+    x = f32_to_bf16_bits((cf[pick] + np.float32(spread) * noise).astype(np.float32))
+    return {"x": x, "centroids": cent, "pick": pick.astype(np.int32)}
