@@ -113,7 +113,7 @@ struct KmeansArgs {
   const uint16_t* x;     // bf16 [M][D], 16-byte aligned rows
   const uint16_t* cent;  // bf16 [C][D]
   int M, C, D;
-  float* hn;             // [C] workspace: |c|^2 / 2
+  float* hn;             // [C] workspace: -|c|^2 / 2
   int32_t* assign;       // [M] (assignment mode)
   float* score;          // [M] or null (assignment mode)
   float* scores;         // [M][C] (score mode)

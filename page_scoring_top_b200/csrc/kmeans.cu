@@ -18,13 +18,14 @@
 //             accumulators of 256 fp32 columns;
 //  * warps 2-9 epilogue, two warpgroups: warpgroup g reads columns
 //             128 g .. 128 g + 127 of each accumulator (each warp its
-//             32-lane quadrant = 32 points), subtracts h, and keeps a
-//             running best per point (h is staged in shared memory by the
-//             same warps, one tile ahead): the maximum of each 32-column chunk
-//             costs one add and one max a column, and only a chunk that beats
-//             the best so far is searched for its first maximal column.  At
-//             the end of a point tile the two halves are combined (the lower
-//             columns win ties) and the assignment (and its score) written.
+//             32-lane quadrant = 32 points), adds -h with paired adds, and
+//             keeps a running best per point (-h is staged in shared memory
+//             by the same warps, one tile ahead): the maximum of each
+//             32-column chunk is a tree of three-input maxima, and only a
+//             chunk that beats the best so far is searched for its first
+//             maximal column.  At the end of a point tile the two halves
+//             are combined (the lower columns win ties) and the assignment
+//             (and its score) written.
 // Score mode writes s[i,c] instead, from the same arithmetic, so an
 // assignment equals the row argmax of the score matrix bit for bit.
 #include <cuda.h>
@@ -60,13 +61,43 @@ struct KmSmem {
   static constexpr size_t tmem_slot = bars + 16 * 8;
   static constexpr size_t misc = tmem_slot + 16;      // abort flag
   static constexpr size_t best = misc + 64;           // [kKmM] value + [kKmM] index, upper half
-  static constexpr size_t hn = 2048;                  // [kKmBStages][kKmN] floats
+  static constexpr size_t hn = 2048;                  // [2][kKmN] floats (by accumulator)
   static constexpr size_t a = 4096;                   // [2] point tiles
   static constexpr size_t b = a + 2 * (size_t)kKmABytes;  // [kKmBStages] centroid tiles
   static constexpr size_t total = b + (size_t)kKmBStages * kKmBBytes + 1024;  // + alignment slack
   static_assert(best + 2 * kKmM * 4 <= hn, "small state overflows");
-  static_assert(hn + (size_t)kKmBStages * kKmN * 4 <= a, "h area overflows");
+  static_assert(hn + 2 * (size_t)kKmN * 4 <= a, "h area overflows");
 };
+
+// x0 += y0, x1 += y1: one paired fp32 add (add.rn.f32x2), each lane rounded
+// to nearest like a scalar add.
+__device__ __forceinline__ void add_pair(float& x0, float& x1, float y0, float y1) {
+  asm("{\n\t.reg .b64 u, v;\n\t"
+      "mov.b64 u, {%0, %1};\n\t"
+      "mov.b64 v, {%2, %3};\n\t"
+      "add.rn.f32x2 u, u, v;\n\t"
+      "mov.b64 {%0, %1}, u;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "f"(y0), "f"(y1));
+}
+
+// The largest of three (a NaN input is ignored, as by fmaxf).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// The largest of 32: three-input maxima 32 -> 11 -> 4 -> 1.
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float t[11];
+#pragma unroll
+  for (int j = 0; j < 10; ++j) t[j] = max3(v[3 * j], v[3 * j + 1], v[3 * j + 2]);
+  t[10] = fmaxf(v[30], v[31]);
+  const float u0 = max3(t[0], t[1], t[2]), u1 = max3(t[3], t[4], t[5]);
+  const float u2 = max3(t[6], t[7], t[8]), u3 = fmaxf(t[9], t[10]);
+  return fmaxf(max3(u0, u1, u2), u3);
+}
 
 // h[c] = (sum_d c[c,d]^2) / 2 in fp32, d in order; one thread per centroid.
 __global__ void kmeans_norms_kernel(const uint16_t* cent, int C, int D, float* hn) {
@@ -84,7 +115,7 @@ __global__ void kmeans_norms_kernel(const uint16_t* cent, int C, int D, float* h
       s = fmaf(hi, hi, s);
     }
   }
-  hn[c] = 0.5f * s;
+  hn[c] = -0.5f * s;  // stored negated: the epilogue adds it
 }
 
 // The main kernel.  SCORES: write s[i,c] to a.scores instead of assigning.
@@ -104,9 +135,9 @@ __global__ void __launch_bounds__(kKmThreads, 1)
   uint64_t* acc_empty = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + KmSmem::tmem_slot);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + KmSmem::misc);
+  float* s_h = reinterpret_cast<float*>(smem + KmSmem::hn);
   float* s_bval = reinterpret_cast<float*>(smem + KmSmem::best);
   int* s_bidx = reinterpret_cast<int*>(smem + KmSmem::best + kKmM * 4);
-  float* s_h = reinterpret_cast<float*>(smem + KmSmem::hn);
   unsigned char* sA = smem + KmSmem::a;
   unsigned char* sB = smem + KmSmem::b;
 
@@ -194,7 +225,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
     const int cbase = wg * (kKmN / 2);
     int i = 0;
     // h of the next centroid tile, loaded a tile ahead (each thread one value)
-    float h_next = (nct > 0 && te < C) ? __ldg(a.hn + te) : 0.f;
+    float h_next = te < C ? __ldg(a.hn + te) : 0.f;
     // (no early exit on abort: every epilogue thread must reach every barrier;
     // after an abort the waits return at once and the loops run out)
     for (int lt = 0; lt < my_tiles; ++lt) {
@@ -215,20 +246,19 @@ __global__ void __launch_bounds__(kKmThreads, 1)
         mbar_wait_bounded(&acc_full[acc], (i >> 1) & 1, s_abort, a.status);
         tc_fence_after();
         const int c0 = n * kKmN + cbase;
-#pragma unroll 1
-        for (int ch = 0; ch < kKmN / 2 / 32; ++ch) {
-          uint32_t raw[32];
-          tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kKmN + cbase + ch * 32),
-                    raw);
+        // 32 columns: subtract h, then (score mode) store, or (assignment)
+        // a tree maximum and, only if it beats the best so far, the first
+        // column that reaches it
+        auto process = [&](const uint32_t (&raw)[32], int ch) {
           float sv[32];
           const float4* h4 = reinterpret_cast<const float4*>(hs + cbase + ch * 32);
 #pragma unroll
           for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 hv = h4[j4];
-            sv[4 * j4 + 0] = __uint_as_float(raw[4 * j4 + 0]) - hv.x;
-            sv[4 * j4 + 1] = __uint_as_float(raw[4 * j4 + 1]) - hv.y;
-            sv[4 * j4 + 2] = __uint_as_float(raw[4 * j4 + 2]) - hv.z;
-            sv[4 * j4 + 3] = __uint_as_float(raw[4 * j4 + 3]) - hv.w;
+            const float4 hv = h4[j4];  // -h
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sv[4 * j4 + q] = __uint_as_float(raw[4 * j4 + q]);
+            add_pair(sv[4 * j4 + 0], sv[4 * j4 + 1], hv.x, hv.y);
+            add_pair(sv[4 * j4 + 2], sv[4 * j4 + 3], hv.z, hv.w);
           }
           const int cc = c0 + ch * 32;  // centroid of sv[0]
           if (SCORES) {
@@ -251,9 +281,7 @@ __global__ void __launch_bounds__(kKmThreads, 1)
               for (int j = 0; j < 32; ++j)
                 if (cc + j >= C) sv[j] = __uint_as_float(kNegInfBits);
             }
-            float mx = sv[0];
-#pragma unroll
-            for (int j = 1; j < 32; ++j) mx = fmaxf(mx, sv[j]);
+            const float mx = max32(sv);
             if (mx > best) {  // strictly: an earlier chunk keeps its ties
               int jj = 31;
 #pragma unroll
@@ -263,28 +291,50 @@ __global__ void __launch_bounds__(kKmThreads, 1)
               bidx = cc + jj;
             }
           }
+        };
+        // two chunks' TMEM loads in flight per wait; the accumulator is free
+        // once the last two are in registers
+        const uint32_t taddr =
+            tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kKmN + cbase);
+        {
+          uint32_t ra[32], rb[32];
+          tmem_ld32_nowait(taddr, ra);
+          tmem_ld32_nowait(taddr + 32, rb);
+          tmem_ld_wait();
+          process(ra, 0);
+          process(rb, 1);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        {
+          uint32_t ra[32], rb[32];
+          tmem_ld32_nowait(taddr + 64, ra);
+          tmem_ld32_nowait(taddr + 96, rb);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          process(ra, 2);
+          process(rb, 3);
+        }
       }
       if (!SCORES) {
-        // the two column halves of every point: the lower half wins ties
+        // the two column halves of every point: the upper half hands its best
+        // to the lower, which keeps its own on ties (lower centroids)
         if (wg == 1) {
           s_bval[row] = best;
           s_bidx[row] = bidx;
         }
         group_sync(kKmEpiWarps * 32);
         if (wg == 0 && point < M) {
-          const float ov = s_bval[row];
-          if (ov > best) {
-            best = ov;
+          const float ob = s_bval[row];
+          if (ob > best) {
+            best = ob;
             bidx = s_bidx[row];
           }
           a.assign[point] = bidx;
           if (a.score) a.score[point] = best;
         }
-        group_sync(kKmEpiWarps * 32);
+        // (the next write of s_bval comes after this tile's readers have
+        // passed the next tile's h barrier)
       }
     }
   }

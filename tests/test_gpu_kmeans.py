@@ -10,7 +10,8 @@ every point to its nearest centroid).
 * against the exact assignment: a chosen centroid's exact score is within
   twice the bound of the best, and the two agree on nearly every point;
 * the full-size workload (262144 points, 1024 centroids, D=128) on sampled
-  points; duplicate centroids go to the lower index; argument errors."""
+  points; duplicate centroids go to the lower index; tiny scores; argument
+  errors."""
 
 import numpy as np
 import pytest
@@ -93,6 +94,21 @@ def test_kmeans_duplicate_centroids_go_low(ctx):
     assign = _check(ctx, d["x"], cent)
     assert not np.any(np.isin(assign, [30, 31, 39]))
     assert np.any(assign == 5)
+
+
+def test_kmeans_tiny_scores(ctx):
+    # inputs scaled by 2^-60: scores near 2^-114, far below the usual range,
+    # with exact ties inside the first 32-column chunk
+    d = synth.kmeans_inputs(91, 500, 300, 128)
+    scale = np.float32(2.0 ** -60)
+
+    def shrink(a):
+        f = (a.astype(np.uint32) << 16).view(np.float32) * scale
+        return (f.view(np.uint32) >> 16).astype(np.uint16)  # exact: a power-of-two scaling
+    x, cent = shrink(d["x"]), shrink(d["centroids"])
+    cent[[7, 8]] = cent[3]  # ties inside the first chunk
+    assign = _check(ctx, x, cent)
+    assert not np.any(np.isin(assign, [7, 8]))
 
 
 def test_kmeans_full_workload_sampled(ctx):
