@@ -67,7 +67,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=("ragged_decode", "prefill_chunk", "causal_decode", "pool_keys",
-                             "paged_decode", "topk_sweep", "kmeans_assign",
+                             "paged_decode", "paged_sweep", "topk_sweep", "kmeans_assign",
                              "batch_decode_bias", "tiny_decode"))
     ap.add_argument("--dists", default="normal,levels16,neg_inf_90",
                     help="top-K sweep distributions (comma list, or 'all')")
@@ -636,8 +636,106 @@ def run_paged(args):
                    "l2": "the 4.2 MB block pool stays in L2; page ids and gathers stream"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
-                     "kernel": "decode_kernel<128,1,fused> (paged producer)"},
+                     "kernel": "decode_tc_kernel<128,16,fused,hist,paged> (tile::gather4 producer)"},
         "gpu_launches": args.steps, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+    }
+    print(json.dumps(line), flush=True)
+    ctx.close()
+    return 0
+
+
+PAGED_REGIMES = ((256, 64), (512, 128), (1024, 256), (2048, 512), (4096, 1024))
+PAGED_BATCHES = (1, 4, 16, 32, 64)
+
+
+def run_paged_sweep(args):
+    """The paged table's own protocol: page counts from five regimes N(256, 64)
+    .. N(4096, 1024) (means doubling, sd a quarter of the mean; counts clipped
+    to 1 .. 2 x mean) x batch {1, 4, 16, 32, 64}, ids uniform over a shared
+    pool of 16384 blocks, head_dim 128, Q = 4.  Each case times
+    centroid_score_paged (score only) and score_topk_fused_paged (K = 256),
+    every call alone with CUDA events after a 256 MB L2 flush (all cases are
+    far below the L2).  Prints one line with every case."""
+    import torch
+    from page_scoring_top_b200 import binding, synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    Q, D, K, NB, seed = 4, 128, 256, 16384, 110
+    peak, peak_src = measured_peak()
+    pool = synth.normal_bf16(seed, 2, 0, NB * D).reshape(NB, D)
+    pd = torch.from_numpy(pool.view(np.int16)).to(dev)
+    nmax = 2 * PAGED_REGIMES[-1][0]
+    ctx = binding.Context(0, max_rows=max(PAGED_BATCHES), max_n=nmax, max_k=K)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    steps = max(3, min(args.steps, 100))
+
+    def time_alone(call):
+        for _ in range(3):
+            call()
+        per = []
+        for _ in range(steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            per.append(e0.elapsed_time(e1))
+        return float(np.median(per))
+
+    cases = []
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.15)
+    for ri, (mu, sd) in enumerate(PAGED_REGIMES):
+        N = 2 * mu
+        for B in PAGED_BATCHES:
+            cs = seed + 10 * ri + PAGED_BATCHES.index(B)
+            z = synth.normal(cs, 0, 0, B)
+            lengths = np.clip(np.round(mu + sd * z), 1, N).astype(np.int32)
+            ids = (synth.u64(cs, 3, 0, B * N) % np.uint64(NB)).astype(np.int32).reshape(B, N)
+            q = synth.normal_bf16(cs, 1, 0, B * Q * D).reshape(B, 1, Q, D)
+            qd = torch.from_numpy(q.view(np.int16)).to(dev)
+            ptd = torch.from_numpy(ids).to(dev)
+            ld = torch.from_numpy(lengths).to(dev)
+            sc = torch.empty((B, 1, N), dtype=torch.float32, device=dev)
+            idx = torch.empty((B, K), dtype=torch.int32, device=dev)
+            ms_s = time_alone(lambda: binding.centroid_score_paged(ctx, qd, pd, ptd, ld, sc,
+                                                                   stream=stream))
+            ms_f = time_alone(lambda: binding.score_topk_fused_paged(ctx, qd, pd, ptd, ld, K, idx,
+                                                                     None, stream=stream))
+            rc, bits = binding.idx_get_status(ctx)
+            if rc != 0:
+                raise RuntimeError("device status %d" % bits)
+            pages = int(lengths.sum())
+            nbytes = pages * (D * 2 + 4) + B * Q * D * 2 + B * 4
+            cases.append({"regime": "N(%d,%d)" % (mu, sd), "B": B, "pages": pages,
+                          "us_score": ms_s * 1e3, "us_fused": ms_f * 1e3,
+                          "pages_per_s_score": pages / (ms_s * 1e-3),
+                          "pages_per_s_fused": pages / (ms_f * 1e-3),
+                          "gbs_score": nbytes / (ms_s * 1e-3) / 1e9})
+    clocks = sampler.stop()
+    head = max(cases, key=lambda c: c["pages"])
+    line = {
+        "metric": "paged pages scored/sec (centroid_score_paged, regime x batch sweep)",
+        "value": head["pages_per_s_score"], "unit": "pages/s", "n_gpus": 1, "steps": steps,
+        "warmup": 3, "ms_per_step": head["us_score"] * 1e-3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "accumulate": "f32",
+        "data": "synthetic",
+        "config": {"workload": "paged_sweep", "Q": Q, "D": D, "K": K, "n_blocks": NB,
+                   "regimes": ["N(%d,%d)" % r for r in PAGED_REGIMES],
+                   "batches": list(PAGED_BATCHES),
+                   "value_case": "%s B=%d" % (head["regime"], head["B"]),
+                   "l2": "flush (256 MB write) before every timed call"},
+        "roofline": {"bound": "hbm", "achieved": head["gbs_score"], "peak": peak, "unit": "GB/s",
+                     "frac": head["gbs_score"] / peak, "traffic": None, "peak_source": peak_src,
+                     "kernel": "decode_tc_kernel<128,16,score,paged> (tile::gather4 producer)"},
+        "geomean_us_score": float(np.exp(np.mean(np.log([c["us_score"] for c in cases])))),
+        "geomean_us_fused": float(np.exp(np.mean(np.log([c["us_fused"] for c in cases])))),
+        "gpu_launches": None, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+        "cases": cases,
     }
     print(json.dumps(line), flush=True)
     ctx.close()
@@ -787,6 +885,8 @@ def main():
         return run_pool(args)
     if args.workload == "paged_decode":
         return run_paged(args)
+    if args.workload == "paged_sweep":
+        return run_paged_sweep(args)
     if args.workload == "topk_sweep":
         return run_topk_sweep(args)
     if args.workload == "kmeans_assign":

@@ -435,10 +435,10 @@ static cudaError_t launch_tt(const DecodeArgs& a, int grid, cudaStream_t stream)
 
 cudaError_t launch_decode(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream) {
   // Head dims 64 and 128 with up to 64 query rows take the tensor-core kernel
-  // (decode_tc.cu), in both modes so that fused and score-mode scores stay
-  // bit-identical; the CUDA-core kernel takes every other shape and every
-  // paged table (its producer copies page by page).
-  if (!a.page_table && decode_tc_supported(a.T, a.Q, a.D, a.ldc_b, a.c))
+  // (decode_tc.cu), contiguous or paged, in both modes so that fused and
+  // score-mode scores stay bit-identical; the CUDA-core kernel takes every
+  // other shape (its paged producer copies page by page).
+  if (decode_tc_supported(a.T, a.Q, a.D, a.page_table ? a.D : a.ldc_b, a.c))
     return launch_decode_tc(a, fused, num_sms, stream);
   const int grid = decode_grid(num_sms);
   if (fused) {

@@ -17,7 +17,10 @@
 //  * warp 8   TMA: 128-page tiles of c (128-byte swizzled, K-major) into a
 //             ring of stages; a segment's ragged tail goes in 32-page boxes.
 //             Up to four lanes issue, stage k by lane k % lanes; L2
-//             evict-first (the centroids are read once).
+//             evict-first (the centroids are read once).  A paged table
+//             (page p of request b = block-pool row page_table[b][p]) is
+//             gathered four rows per copy (tile::gather4), the whole warp
+//             filling each tile.
 //  * warp 9   MMA: writes the request's query rows into the B operand when
 //             the request changes, then one thread issues D/16 tcgen05.mma
 //             (M128, N = T*Q rounded up to 16, K16) per tile into one of four
@@ -110,8 +113,10 @@ __host__ __device__ inline TcLayout tc_layout(bool fused, int D, int T, int Q) {
 }
 
 // D: head dim (64 or 128).  NC: query rows the epilogue unrolls (16 or 64).
-// HIST: single-token fused rows with the histogram select.
-template <int D, int NC, bool FUSED, bool HIST>
+// HIST: single-token fused rows with the histogram select.  PAGED: page p of
+// request b is row page_table[b][p] of a block pool (map_tile is then the
+// pool as [n_blocks][D] with one-row boxes, and map_sub is unused).
+template <int D, int NC, bool FUSED, bool HIST, bool PAGED>
 __global__ void __launch_bounds__(kTcThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap map_tile,
                      const __grid_constant__ CUtensorMap map_sub, const DecodeArgs a) {
@@ -183,7 +188,66 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const Chunking ch = make_chunking(s_off, B, G, FUSED ? kSegmentPages : 0, FUSED ? kTcLMin : 1);
   const int nchunks = ch.nchunks;
 
-  if (warp == kTcProducerWarp) {
+  if (PAGED && warp == kTcProducerWarp) {
+    // ------------------------------------------------------------ TMA gather producer
+    // The whole warp fills each tile: lane i reads the block ids of pages
+    // 4i .. 4i+3 of the tile and gathers the four pool rows per 64-column K
+    // block (tile::gather4), which land where a tile load of those rows would
+    // put them.  A last group past the segment end repeats its first page.
+    // Ids outside the pool are clamped and reported.  No L2 hint: pool rows
+    // are shared across requests and stay hot.
+    uint32_t tile = 0;
+    int64_t last = -1;  // last tile this warp filled
+    for (int j = g; j < nchunks; j += G) {
+      const int cb = ch.chunk_begin(j), ce = ch.chunk_end(j);
+      const int b_last = ch.row(ce - 1);
+      for (int b = ch.row(cb); b <= b_last; ++b) {
+        if (ch.len(b) == 0) continue;
+        const int p0 = ch.snap(b, cb);
+        const int nps = ch.snap(b, ce) - p0;
+        const int32_t* pt = a.page_table + (int64_t)b * a.ld_pt + p0;
+        for (int r0 = 0; r0 < nps; r0 += kTcTile, ++tile) {
+          const int slot = (int)(tile % (uint32_t)nst);
+          const uint32_t round = tile / (uint32_t)nst;
+          int go = 1;
+          if (lane == 0) {
+            if (round > 0) mbar_wait_bounded(&empty[slot], (round - 1) & 1, s_abort, a.status);
+            go = *s_abort == 0;
+          }
+          go = __shfl_sync(0xFFFFFFFFu, go, 0);
+          if (!go) continue;
+          const int rem = min(kTcTile, nps - r0);
+          const int ngr = (rem + 3) >> 2;  // 4-row groups
+          if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)ngr * 4u * 128u * KB);
+          __syncwarp();
+          if (lane < ngr) {
+            int y[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int r = 4 * lane + u;
+              int blk = __ldg(pt + r0 + (r < rem ? r : 4 * lane));
+              if (blk < 0 || blk >= a.n_blocks) {
+                atomicOr(a.status, kErrPageClamped);
+                blk = blk < 0 ? 0 : a.n_blocks - 1;
+              }
+              y[u] = blk;
+            }
+            unsigned char* dst = ring + (size_t)slot * stage_bytes + (size_t)lane * 4 * 128;
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb)
+              tma_gather4(dst + kb * kBlock, &map_tile, kb * 64, y[0], y[1], y[2], y[3],
+                          &full[slot]);
+          }
+          last = tile;
+        }
+      }
+    }
+    // Nothing may still be landing in shared memory when the CTA exits (this
+    // matters only after an abort): wait for the last tiles' copies.
+    if (lane == 0)
+      for (int64_t t = last; t >= 0 && t > last - nst; --t)
+        mbar_wait_drain(&full[t % nst], (uint32_t)(t / nst) & 1);
+  } else if (warp == kTcProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     const int lanes = L.lanes;
     if (lane < lanes) {
@@ -406,10 +470,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template <int D, int NC, bool FUSED, bool HIST>
+template <int D, int NC, bool FUSED, bool HIST, bool PAGED>
 cudaError_t launch_tc(const CUtensorMap& mt, const CUtensorMap& ms, const DecodeArgs& a, int grid,
                       size_t smem, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NC, FUSED, HIST>,
+  cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, NC, FUSED, HIST, PAGED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Launched as a programmatic dependent of the previous kernel in the
@@ -424,14 +488,22 @@ cudaError_t launch_tc(const CUtensorMap& mt, const CUtensorMap& ms, const Decode
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<D, NC, FUSED, HIST>, mt, ms, a);
+  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<D, NC, FUSED, HIST, PAGED>, mt, ms, a);
 }
 
-template <int D, bool FUSED, bool HIST>
+template <int D, bool FUSED, bool HIST, bool PAGED>
 cudaError_t launch_nc(const CUtensorMap& mt, const CUtensorMap& ms, const DecodeArgs& a, int grid,
                       size_t smem, cudaStream_t stream) {
-  if (a.T * a.Q <= 16) return launch_tc<D, 16, FUSED, HIST>(mt, ms, a, grid, smem, stream);
-  return launch_tc<D, 64, FUSED, HIST>(mt, ms, a, grid, smem, stream);
+  if (a.T * a.Q <= 16) return launch_tc<D, 16, FUSED, HIST, PAGED>(mt, ms, a, grid, smem, stream);
+  return launch_tc<D, 64, FUSED, HIST, PAGED>(mt, ms, a, grid, smem, stream);
+}
+
+template <int D, bool PAGED>
+cudaError_t launch_modes(const CUtensorMap& mt, const CUtensorMap& ms, const DecodeArgs& a,
+                         bool fused, int grid, size_t smem, cudaStream_t stream) {
+  if (!fused) return launch_nc<D, false, false, PAGED>(mt, ms, a, grid, smem, stream);
+  if (a.T == 1) return launch_nc<D, true, true, PAGED>(mt, ms, a, grid, smem, stream);
+  return launch_nc<D, true, false, PAGED>(mt, ms, a, grid, smem, stream);
 }
 
 }  // namespace
@@ -444,9 +516,27 @@ bool decode_tc_supported(int T, int Q, int D, int64_t ldc_b, const void* c) {
 }
 
 cudaError_t launch_decode_tc(const DecodeArgs& a, bool fused, int num_sms, cudaStream_t stream) {
-  if (!decode_tc_supported(a.T, a.Q, a.D, a.ldc_b, a.c)) return cudaErrorNotSupported;
+  if (!decode_tc_supported(a.T, a.Q, a.D, a.page_table ? a.D : a.ldc_b, a.c))
+    return cudaErrorNotSupported;
   auto encode = get_encode();
   if (!encode) return cudaErrorNotSupported;
+  const TcLayout L = tc_layout(fused, a.D, a.T, a.Q);
+  const int grid = num_sms;
+  if (a.page_table) {
+    // the block pool as [n_blocks][D] bf16; one-row boxes of 64 columns
+    // (128 B, 128-byte swizzle) for the four-row gathers
+    CUtensorMap mp;
+    const cuuint64_t dims[2] = {(cuuint64_t)a.D, (cuuint64_t)a.n_blocks};
+    const cuuint64_t strides[1] = {(cuuint64_t)a.D * 2};
+    const cuuint32_t estr[2] = {1, 1};
+    const cuuint32_t box[2] = {64, 1};
+    if (encode(&mp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.c), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    if (a.D == 128) return launch_modes<128, true>(mp, mp, a, fused, grid, L.total, stream);
+    return launch_modes<64, true>(mp, mp, a, fused, grid, L.total, stream);
+  }
   // c as [B][N][D] bf16 with request stride ldc_b; boxes of 64 columns (128 B,
   // 128-byte swizzle) x 128 pages (whole tiles) or x 32 pages (ragged tails)
   CUtensorMap mt, ms;
@@ -463,17 +553,8 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, bool fused, int num_sms, cudaS
              box_s, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const TcLayout L = tc_layout(fused, a.D, a.T, a.Q);
-  const int grid = num_sms;
-  const bool hist = fused && a.T == 1;
-  if (a.D == 128) {
-    if (!fused) return launch_nc<128, false, false>(mt, ms, a, grid, L.total, stream);
-    if (hist) return launch_nc<128, true, true>(mt, ms, a, grid, L.total, stream);
-    return launch_nc<128, true, false>(mt, ms, a, grid, L.total, stream);
-  }
-  if (!fused) return launch_nc<64, false, false>(mt, ms, a, grid, L.total, stream);
-  if (hist) return launch_nc<64, true, true>(mt, ms, a, grid, L.total, stream);
-  return launch_nc<64, true, false>(mt, ms, a, grid, L.total, stream);
+  if (a.D == 128) return launch_modes<128, false>(mt, ms, a, fused, grid, L.total, stream);
+  return launch_modes<64, false>(mt, ms, a, fused, grid, L.total, stream);
 }
 
 }  // namespace idx

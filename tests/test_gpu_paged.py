@@ -100,3 +100,33 @@ def test_paged_out_of_range_entry_is_clamped_and_reported(ctx):
     keep = np.arange(64) != 5
     assert oracle.score_bound_violations(s_gpu[..., keep], S[..., keep], A[..., keep]) == 0
     assert np.isfinite(s_gpu[0, 0, 5])
+
+
+@pytest.mark.parametrize("D,lengths", [(128, [4096, 37, 4000, 129, 1]), (64, [2048, 2047, 5, 0])])
+def test_paged_equals_gathered_table(ctx, D, lengths):
+    # The same centroids as a contiguous per-request table (pool rows gathered
+    # on the host): both calls run the same tensor-core arithmetic, so scores
+    # and selections are bit-identical; ragged tails exercise the partial
+    # four-row gathers.
+    from page_scoring_top_b200 import binding
+    B = len(lengths)
+    N = max(lengths)
+    q, pool, pt, ln = _inputs(940 + D, B, 1, 4, D, N, 3000, lengths)
+    c = pool[pt]  # [B][N][D]
+    qd, ld = to_dev_bf16(q), to_dev(ln)
+    s_pg = torch.empty((B, 1, N), device="cuda")
+    s_ct = torch.empty((B, 1, N), device="cuda")
+    binding.centroid_score_paged(ctx, qd, to_dev_bf16(pool), to_dev(pt), ld, s_pg)
+    binding.centroid_score(ctx, qd, to_dev_bf16(c), ld, s_ct)
+    K = 128
+    i_pg, v_pg = poisoned_outputs(B, K)
+    i_ct, v_ct = poisoned_outputs(B, K)
+    binding.score_topk_fused_paged(ctx, qd, to_dev_bf16(pool), to_dev(pt), ld, K, i_pg, v_pg)
+    binding.score_topk_fused(ctx, qd, to_dev_bf16(c), ld, K, i_ct, v_ct)
+    rc, bits = binding.idx_get_status(ctx)
+    assert rc == 0 and bits == 0
+    for b, n in enumerate(lengths):
+        assert np.array_equal(s_pg.cpu().numpy()[b, 0, :n].view(np.int32),
+                              s_ct.cpu().numpy()[b, 0, :n].view(np.int32))
+    assert np.array_equal(i_pg.cpu().numpy(), i_ct.cpu().numpy())
+    assert np.array_equal(v_pg.cpu().numpy().view(np.int32), v_ct.cpu().numpy().view(np.int32))
