@@ -82,7 +82,7 @@ __host__ __device__ inline DecodeLayout decode_layout(bool fused, int D, int T) 
   L.hist = o;  // single-token filters also keep their digit histograms
   o += (fused && T == 1) ? (size_t)(kHBins + kHCoarse) * 4 : 0;
   L.off = o;
-  o += align16((size_t)(kDecodeMaxB + 1) * 4);
+  o += align16((size_t)(kDecodeMaxB + 2) * 4);  // prefix sums + the longest length
   L.bar = o;
   o += (size_t)2 * kMaxStages * 8;
   L.misc = o;
@@ -162,7 +162,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) decode_kernel(const DecodeA
   }
   length_prefix(a, s_off, s_wsum, kDecodeThreads);
   __syncthreads();
-  const Chunking ch = make_chunking(s_off, B, G, FUSED ? kSegmentPages : 0, FUSED ? kLMin : 1);
+  const Chunking ch = FUSED ? make_fused_chunking(s_off, B, G, kSegmentPages, kLMin, a.K)
+                            : make_chunking(s_off, B, G, 0, 1);
   const int nchunks = ch.nchunks;
 
   // ------------------------------------------------------------------ producer

@@ -80,7 +80,7 @@ __host__ __device__ inline TcLayout tc_layout(bool fused, int D, int T, int Q) {
   L.misc = o;  // abort, flag, TMEM base, warp sums
   o += 64;
   L.off = o;
-  o += al16((size_t)(kDecodeMaxB + 1) * 4);
+  o += al16((size_t)(kDecodeMaxB + 2) * 4);  // prefix sums + the longest length
   L.fbuf = o;
   o += fused ? (size_t)kFilterCap * 8 : 0;
   L.fstate = o;
@@ -185,7 +185,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const Chunking ch = make_chunking(s_off, B, G, FUSED ? kSegmentPages : 0, FUSED ? kTcLMin : 1);
+  const Chunking ch = FUSED ? make_fused_chunking(s_off, B, G, kSegmentPages, kTcLMin, a.K)
+                            : make_chunking(s_off, B, G, 0, 1);
   const int nchunks = ch.nchunks;
 
   if (PAGED && warp == kTcProducerWarp) {

@@ -19,6 +19,7 @@
 namespace idx {
 
 constexpr int kSelThreads = 256;  // threads 0..255 run every select step
+static_assert(2 * (kSelThreads / 32) <= 32, "per-warp key maxima and minima fit the scratch");
 constexpr int kMaxFusedT = 4;
 // Virtual pages charged per request in fused mode: about what a segment-end
 // select step costs in streaming time (a few microseconds at one SM's share
@@ -201,7 +202,7 @@ static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, 
     sc.ctr = 0;
     if (single) *row_thr = 0ull;  // raised while streaming, read by nobody else
   }
-  if (single) fine_clear<kSelThreads>(ar);
+  fine_clear<kSelThreads>(ar);
   const int nk = load_buffer<kSelThreads, E>(fb, fi, fs.count, v, bits);
   IDX_TRACE(19);
   group_sync(kSelThreads);
@@ -212,11 +213,26 @@ static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, 
   const uint64_t vpub = (uint64_t)bp << (32 + kHShift);
   IDX_TRACE(13);
   bool ok = true;
+  const uint32_t khi = bmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((bmax + 1) << kHShift) - 1u;
   if (single) {
-    const uint32_t khi =
-        bmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((bmax + 1) << kHShift) - 1u;
     ok = fine_select<kSelThreads, E>(v, bits, nk, vlo, khi, o.K, ar, out_emit, out_pad);
-  } else if (n0 <= (uint32_t)lcap) {
+  } else if (n0 > (uint32_t)lcap) {
+    // more entries at or above the publish floor than a list holds (the
+    // boundary digit is wide): publish the segment's exact top K instead
+    auto pub_emit = [&](int pos, uint64_t x, uint32_t xb) {
+      cbits[pos] = xb;
+      cidx[pos] = (int32_t)~(uint32_t)x;
+    };
+    auto pub_pad = [&](int pos) {
+      cbits[pos] = kNegInfBits;
+      cidx[pos] = -1;
+    };
+    ok = fine_select<kSelThreads, E>(v, bits, nk, vlo, khi, o.K, ar, pub_emit, pub_pad);
+    if (ok) {
+      for (int p = o.K + (int)threadIdx.x; p < lcap; p += kSelThreads) pub_pad(p);
+      if (threadIdx.x == 0 && b0 != 0) atomicMax(row_thr, (unsigned long long)vlo);
+    }
+  } else {
 #pragma unroll
     for (int k = 0; k < E; ++k)
       if (k < nk && v[k] >= vpub && v[k] != 0) {
@@ -230,8 +246,6 @@ static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, 
     }
     // with b0 > 0 the segment holds K entries >= vlo: so does its row
     if (threadIdx.x == 0 && b0 != 0) atomicMax(row_thr, (unsigned long long)vlo);
-  } else {
-    ok = false;
   }
   if (!ok) {
     // a crowded digit bin (heavy ties): exact radix compaction first
@@ -258,11 +272,24 @@ static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, 
                                fb, fi);
       IDX_TRACE(25);
       const int nkm = load_buffer<kSelThreads, E>(fb, fi, nslots * lcap, v, bits);
-      uint32_t km = 0;
+      // The fine select over the candidates' key span, floored by the
+      // request's threshold: with a threshold raised by the segments the span
+      // is narrow.  When it is not (short segments) or the boundary bin is
+      // crowded all the same, the candidates' own digit histogram bounds the
+      // K-th largest as a segment's does, and the fine select runs again over
+      // the digits from there up.
+      uint32_t km = 0, kn = 0xFFFFFFFFu;
 #pragma unroll
-      for (int k = 0; k < E; ++k) km = max(km, (uint32_t)(v[k] >> 32));
+      for (int k = 0; k < E; ++k) {
+        km = max(km, (uint32_t)(v[k] >> 32));
+        if (v[k] != 0) kn = min(kn, (uint32_t)(v[k] >> 32));
+      }
       km = __reduce_max_sync(0xFFFFFFFFu, km);
-      if (lane_id() == 0) sc.wsum[threadIdx.x >> 5] = km;
+      kn = __reduce_min_sync(0xFFFFFFFFu, kn);
+      if (lane_id() == 0) {
+        sc.wsum[threadIdx.x >> 5] = km;
+        sc.wsum[kSelThreads / 32 + (threadIdx.x >> 5)] = kn;
+      }
       if (threadIdx.x == 0) {
         *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = __ldcg(row_thr);
         *row_thr = 0ull;  // zero for the next call
@@ -270,11 +297,40 @@ static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, 
       fine_clear<kSelThreads>(ar);
       group_sync(kSelThreads);
       IDX_TRACE(26);
-      const uint64_t thr = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
       km = 0;
+      kn = 0xFFFFFFFFu;
 #pragma unroll
-      for (int w = 0; w < kSelThreads / 32; ++w) km = max(km, sc.wsum[w]);
-      done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, o.K, ar, out_emit, out_pad);
+      for (int w = 0; w < kSelThreads / 32; ++w) {
+        km = max(km, sc.wsum[w]);
+        kn = min(kn, sc.wsum[kSelThreads / 32 + w]);
+      }
+      const uint64_t thr0 = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
+      uint64_t thr = thr0 > ((uint64_t)kn << 32) ? thr0 : ((uint64_t)kn << 32);
+      // (every thread has read wsum and bcast before fine_select's first barrier)
+      if (thr0 != 0)
+        done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, o.K, ar, out_emit, out_pad);
+      if (!done) {
+        // (the segment's digit histogram is spent: the next segment clears it)
+        hist_clear<kSelThreads>(f.hist, f.hist + kHBins);
+        group_sync(kSelThreads);
+#pragma unroll
+        for (int k = 0; k < E; ++k)
+          if (k < nkm && v[k] >= thr0 && v[k] != 0) {
+            const uint32_t d = (uint32_t)(v[k] >> (32 + kHShift));
+            atomicAdd(&f.hist[d], 1u);
+            atomicAdd(&f.hist[kHBins + (d >> 5)], 1u);
+          }
+        group_sync(kSelThreads);
+        if ((threadIdx.x >> 5) == 0)
+          warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)o.K, 0u, sc.bcast);
+        group_sync(kSelThreads);
+        const uint32_t mb0 = sc.bcast[0], mbmax = sc.bcast[1];
+        const uint64_t mlo = (uint64_t)mb0 << (32 + kHShift);
+        thr = thr0 > mlo ? thr0 : mlo;
+        const uint32_t mhi =
+            mbmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((mbmax + 1) << kHShift) - 1u;
+        done = fine_select<kSelThreads, E>(v, bits, nkm, thr, mhi, o.K, ar, out_emit, out_pad);
+      }
       if (!done) {
         // a crowded boundary bin (heavy ties): the entries at or above the
         // threshold go back to the buffer for the exact radix compaction
@@ -400,7 +456,10 @@ __device__ __forceinline__ void length_prefix(const DecodeArgs& a, int* s_off, u
                                               int nthreads) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int running = 0;
-  if (tid == 0) s_off[0] = 0;
+  if (tid == 0) {
+    s_off[0] = 0;
+    s_off[a.B + 1] = 0;  // the longest (clamped) length
+  }
   for (int base = 0; base < a.B; base += nthreads) {
     const int i = base + tid;
     int len = 0;
@@ -416,8 +475,10 @@ __device__ __forceinline__ void length_prefix(const DecodeArgs& a, int* s_off, u
       }
     }
     const uint32_t incl = warp_incl_scan((uint32_t)len);
+    const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, (uint32_t)len);
     if (lane == 31) s_wsum[warp] = incl;
     __syncthreads();
+    if (lane == 0) atomicMax(&s_off[a.B + 1], (int)wmax);
     uint32_t excl = incl - (uint32_t)len, total = 0;
     for (int w = 0; w < nthreads / 32; ++w) {
       if (w < warp) excl += s_wsum[w];
@@ -488,6 +549,19 @@ __device__ __forceinline__ Chunking make_chunking(const int* s_off, int B, int G
   c.Lc = Lc < 1 ? 1 : Lc;
   c.nchunks = (c.PV + c.Lc - 1) / c.Lc;
   return c;
+}
+
+// The work split of a fused launch: chunks of at least `lmin` pages, and
+// long enough that no request is cut into more segments than the merge
+// stages at once (kFilterCap entries, at least K from each segment): a
+// request of L pages spans at most ceil(L / Lc) + 1 chunks.  s_off[B + 1]
+// holds the longest length (length_prefix).
+__device__ __forceinline__ Chunking make_fused_chunking(const int* s_off, int B, int G, int W,
+                                                        int lmin, int K) {
+  int smax = kFilterCap / ((K + 3) & ~3);
+  smax = smax < 2 ? 2 : smax;
+  const int lk = (s_off[B + 1] + smax - 2) / (smax - 1);
+  return make_chunking(s_off, B, G, W, lmin > lk ? lmin : lk);
 }
 
 }  // namespace idx
