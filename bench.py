@@ -51,6 +51,7 @@ FALLBACK_HBM_GBS = 6650.0
 # The ncu summary of the headline kernel records its DRAM bytes per valid page
 # beside a digest of the library sources it was captured on; the traffic is
 # reported only while the sources still have that digest.
+L2_BYTES = 126 << 20
 TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "decode_fused_ragged_decode.md")
 REPEATS = 11  # timed regions of exactly --steps steps; the median is reported
 
@@ -71,6 +72,11 @@ def parse():
                              "batch_decode_bias", "tiny_decode"))
     ap.add_argument("--dists", default="normal,levels16,neg_inf_90",
                     help="top-K sweep distributions (comma list, or 'all')")
+    ap.add_argument("--topk-case", default=None,
+                    help="top-K sweep: only the rows x N case given as ROWSxN (e.g. 128x262144)")
+    ap.add_argument("--head-dim", type=int, default=None,
+                    help="decode workloads: override D (64 and 128 take the tensor-core "
+                         "kernel, other multiples of 8 the CUDA-core one)")
     return ap.parse_args()
 
 
@@ -81,12 +87,13 @@ def dist_env():
     return rank, world, local
 
 
-def workload_inputs(rank, name=WORKLOAD):
+def workload_inputs(rank, name=WORKLOAD, head_dim=None):
     from page_scoring_top_b200 import dist as pdist
     from page_scoring_top_b200 import synth
     spec = dict(synth.WORKLOADS[name])
     seed = pdist.rank_seed(spec["seed"], rank)
-    return synth.workload(name, seed=seed), spec, seed
+    over = {} if head_dim is None else {"D": head_dim}
+    return synth.workload(name, seed=seed, **over), spec, seed
 
 
 def algorithmic_bytes(lengths, B, T, Q, D, K, with_values):
@@ -332,7 +339,7 @@ def run_ours(args):
         pg = dist
     from page_scoring_top_b200 import binding
 
-    d, spec, seed = workload_inputs(rank, args.workload)
+    d, spec, seed = workload_inputs(rank, args.workload, args.head_dim)
     B, T, Q, D = d["q"].shape
     N = d["c"].shape[1]
     K = spec["K"]
@@ -350,11 +357,23 @@ def run_ours(args):
     ctx = binding.Context(local, max_rows=B * T, max_n=N, max_k=K)
     stream = torch.cuda.current_stream(dev)
 
+    # A centroid table below the L2 is replicated until the copies exceed
+    # twice the L2, and the steps rotate over them: every step reads inputs
+    # that are not L2-resident, back to back.
+    small = c.numel() * 2 < L2_BYTES
+    copies = [(q, c)]
+    if small:
+        ncopy = -(-2 * L2_BYTES // (c.numel() * 2))
+        copies += [(q.clone(), c.clone()) for _ in range(ncopy - 1)]
+    turn = [0]
+
     def step():
+        qq, cc = copies[turn[0] % len(copies)]
+        turn[0] += 1
         if tokd is not None:
-            binding.score_topk_fused_tokens(ctx, q, c, tokd, K, idx, None, stream=stream)
+            binding.score_topk_fused_tokens(ctx, qq, cc, tokd, K, idx, None, stream=stream)
         else:
-            binding.score_topk_fused(ctx, q, c, ln, K, idx, None, stream=stream)
+            binding.score_topk_fused(ctx, qq, cc, ln, K, idx, None, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -400,7 +419,9 @@ def run_ours(args):
     # kernel (centroid_score alone) is timed the same way on the same stream.
     peak, peak_src = measured_peak()
     kernel, traffic, traffic_note = KERNEL, None, "no ncu capture for this workload"
-    if args.workload == WORKLOAD:
+    if args.head_dim is not None and args.head_dim not in (64, 128):
+        kernel = "decode_kernel<D=%d,fused> (CUDA cores)" % args.head_dim
+    elif args.workload == WORKLOAD and args.head_dim is None:
         per_page, traffic_note = recorded_traffic_per_page()
         traffic = None if per_page is None else per_page * pages
     launch_s = (ms / args.steps) * 1e-3
@@ -451,8 +472,12 @@ def run_ours(args):
                                     else "all pages valid"), "seed": seed,
                        "pages_per_step_per_gpu": pages, "bytes_per_step_per_gpu": nbytes,
                        "parallelism": "dp%d (requests sharded, no data-path collective)" % world,
-                       "l2": "inputs larger than L2 (%.1f MB of centroids per step vs 126 MB); "
-                             "no flush" % (pages * D * 2 / 1e6)},
+                       "l2": ("centroid table of %.1f MB is below the 126 MB L2: the steps "
+                              "rotate over %d copies of q and c (%.0f MB), back to back"
+                              % (c.numel() * 2 / 1e6, len(copies),
+                                 len(copies) * c.numel() * 2 / 1e6)) if small else
+                             ("inputs larger than L2 (%.1f MB of centroids per step vs 126 MB); "
+                              "no flush" % (pages * D * 2 / 1e6))},
             "hbm_gbs": achieved, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "traffic_source": traffic_note,
@@ -765,8 +790,9 @@ def run_topk_sweep(args):
     sampler = ClockSampler(0)
     sampler.start()
     time.sleep(0.15)
+    only = None if args.topk_case is None else tuple(int(x) for x in args.topk_case.split("x"))
     for case, rows, n, dist in synth.sweep_cases():
-        if dist not in dists:
+        if dist not in dists or (only is not None and (rows, n) != only):
             continue
         s = torch.from_numpy(synth.score_rows(104 + case, rows, n, dist)).to(dev)
         idx = torch.empty((rows, K), dtype=torch.int32, device=dev)
