@@ -41,11 +41,14 @@ struct FusedSel {
   uint32_t* s_row;
 };
 
-// Filter entries per token for T tokens.
-__host__ __device__ inline int fused_cap(int T) {
+// Filter entries per token for T tokens, the buffer holding `bufs` x
+// kFilterCap entries in all (at most kFilterCap per token: a filter is
+// loaded into registers whole).
+__host__ __device__ inline int fused_cap(int T, int bufs = 1) {
   int tp = 1;
   while (tp < T) tp <<= 1;
-  return kFilterCap / tp;
+  const int c = bufs * kFilterCap / tp;
+  return c < kFilterCap ? c : kFilterCap;
 }
 
 // Segment start (all select threads; the caller syncs after).
@@ -147,6 +150,130 @@ struct RowOut {
   int32_t* arrive;              // per row, zero between calls
 };
 
+// The merge of a request row's published lists by the last CTA to arrive,
+// when they fit the filter buffer together (nslots * lcap <= kFilterCap; every
+// filter of the CTA is spent): the lists are staged into the buffer, then the
+// fine select runs over the candidates' key span floored by the row's
+// threshold.  When no threshold was raised or the boundary bin is crowded, the
+// candidates' own digit histogram (in `dhist`, kHBins + kHCoarse words; null
+// to skip this step) bounds the K-th largest first; heavy ties go to the
+// radix compaction.  Writes the row, resets *row_thr.  All select threads.
+template <class SlotOf>
+__device__ bool merge_staged(const FusedSel& f, int nslots, SlotOf slot_of, const uint32_t* cand_bits,
+                             const int32_t* cand_idx, int64_t stride, int lcap, int K,
+                             unsigned long long* row_thr, uint32_t* dhist, int32_t* out_i,
+                             float* out_v) {
+  SelectScratch& sc = *f.sc;
+  FilterState& fs = f.fst[0];
+  uint32_t* fb = f.fbuf;
+  uint32_t* fi = f.fbuf + kFilterCap;
+  uint32_t* fine = &sc.hist[1][0];
+  const FineArea ar{fine,    fine + kFineBins, f.sortv, f.sortb,
+                    reinterpret_cast<uint64_t*>(f.fbuf), f.fbuf + 2 * (kFineBoundaryMax + 2),
+                    sc.wsum, sc.bcast};
+  constexpr int E = kFilterCap / kSelThreads;
+  uint64_t v[E];
+  uint32_t bits[E];
+  auto out_emit = [&](int pos, uint64_t x, uint32_t xb) {
+    out_i[pos] = (int32_t)~(uint32_t)x;
+    if (out_v) out_v[pos] = __uint_as_float(xb);
+  };
+  auto out_pad = [&](int pos) {
+    out_i[pos] = -1;
+    if (out_v) out_v[pos] = __uint_as_float(kNegInfBits);
+  };
+  bool done = false;
+  // the request's final threshold, read while the lists are staged
+  unsigned long long rt = 0ull;
+  if (threadIdx.x == 0) {
+    rt = __ldcg(row_thr);
+    *row_thr = 0ull;  // zero for the next call
+  }
+  // the buffer (already published) receives every list
+  stage_lists<kSelThreads>(nslots, slot_of, cand_bits, cand_idx, stride, lcap, fb, fi);
+  IDX_TRACE(25);
+  const int nkm = load_buffer<kSelThreads, E>(fb, fi, nslots * lcap, v, bits);
+  // The fine select over the candidates' key span, floored by the
+  // request's threshold: with a threshold raised by the segments the span
+  // is narrow.  When it is not (short segments) or the boundary bin is
+  // crowded all the same, the candidates' own digit histogram bounds the
+  // K-th largest as a segment's does, and the fine select runs again over
+  // the digits from there up.
+  uint32_t km = 0, kn = 0xFFFFFFFFu;
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    km = max(km, (uint32_t)(v[k] >> 32));
+    if (v[k] != 0) kn = min(kn, (uint32_t)(v[k] >> 32));
+  }
+  km = __reduce_max_sync(0xFFFFFFFFu, km);
+  kn = __reduce_min_sync(0xFFFFFFFFu, kn);
+  if (lane_id() == 0) {
+    sc.wsum[threadIdx.x >> 5] = km;
+    sc.wsum[kSelThreads / 32 + (threadIdx.x >> 5)] = kn;
+  }
+  if (threadIdx.x == 0) *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = rt;
+  fine_clear<kSelThreads>(ar);
+  group_sync(kSelThreads);
+  IDX_TRACE(26);
+  km = 0;
+  kn = 0xFFFFFFFFu;
+#pragma unroll
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    km = max(km, sc.wsum[w]);
+    kn = min(kn, sc.wsum[kSelThreads / 32 + w]);
+  }
+  const uint64_t thr0 = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
+  uint64_t thr = thr0 > ((uint64_t)kn << 32) ? thr0 : ((uint64_t)kn << 32);
+  // (every thread has read wsum and bcast before fine_select's first barrier)
+  if (thr0 != 0 || !dhist)
+    done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, K, ar, out_emit, out_pad);
+  if (!done && dhist) {
+    // (a spent digit histogram: the next segment clears it)
+    hist_clear<kSelThreads>(dhist, dhist + kHBins);
+    group_sync(kSelThreads);
+#pragma unroll
+    for (int k = 0; k < E; ++k)
+      if (k < nkm && v[k] >= thr0 && v[k] != 0) {
+        const uint32_t d = (uint32_t)(v[k] >> (32 + kHShift));
+        atomicAdd(&dhist[d], 1u);
+        atomicAdd(&dhist[kHBins + (d >> 5)], 1u);
+      }
+    group_sync(kSelThreads);
+    if ((threadIdx.x >> 5) == 0)
+      warp_hist_bounds(dhist, dhist + kHBins, (uint32_t)K, 0u, sc.bcast);
+    group_sync(kSelThreads);
+    const uint32_t mb0 = sc.bcast[0], mbmax = sc.bcast[1];
+    const uint64_t mlo = (uint64_t)mb0 << (32 + kHShift);
+    thr = thr0 > mlo ? thr0 : mlo;
+    const uint32_t mhi =
+        mbmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((mbmax + 1) << kHShift) - 1u;
+    done = fine_select<kSelThreads, E>(v, bits, nkm, thr, mhi, K, ar, out_emit, out_pad);
+  }
+  if (!done) {
+    // a crowded boundary bin (heavy ties): the entries at or above the
+    // threshold go back to the buffer for the exact radix compaction
+    if (threadIdx.x == 0) sc.ctr = 0;
+    group_sync(kSelThreads);
+#pragma unroll
+    for (int k = 0; k < E; ++k)
+      if (k < nkm && v[k] >= thr && v[k] != 0) {
+        const int p = atomicAdd(&sc.ctr, 1);
+        fb[p] = bits[k];
+        fi[p] = ~(uint32_t)v[k];
+      }
+    group_sync(kSelThreads);
+    if (threadIdx.x == 0) {
+      fs.count = sc.ctr;
+      fs.thr = 0ull;
+    }
+    group_sync(kSelThreads);
+    filter_compact<kSelThreads>(fs, fb, fi, K, sc);
+    sort_and_write<kSelThreads>(fb, fi, fs.count, K, f.sortv, f.sortb, out_i, out_v);
+    done = true;
+  }
+  return done;
+}
+
 // Segment end of single-token row b in chunk j, the row spanning chunks
 // j0..j1 (all select threads, after a barrier that completed every offer).
 // The filter's digit histogram is exact for its buffer: one warp reads from
@@ -192,9 +319,9 @@ static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, 
     out_i[pos] = -1;
     if (out_v) out_v[pos] = __uint_as_float(kNegInfBits);
   };
-  // Every asynchronous poll of the request's threshold has landed (the
-  // next segment may belong to another request).
-  cp_async_wait_all();
+  // (A poll of the request's threshold may still be landing in s_row: either
+  // value is a floor of this request's K-th largest.  The wait for it comes
+  // at the end, before the next segment resets s_row.)
   if ((threadIdx.x >> 5) == 0)
     warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)o.K, single ? 0u : *f.s_row >> kHShift,
                      sc.bcast);
@@ -266,100 +393,18 @@ static __device__ void hist_finalize(const FusedSel& f, const RowOut& o, int b, 
     IDX_TRACE(15);
     auto slot_of = [=](int i) { return (int64_t)(j0 + i + b); };
     bool done = false;
-    if (nslots * lcap <= kFilterCap) {
-      // the buffer (already published) receives every list
-      stage_lists<kSelThreads>(nslots, slot_of, o.cand_bits, o.cand_idx, o.slot_stride, lcap,
-                               fb, fi);
-      IDX_TRACE(25);
-      const int nkm = load_buffer<kSelThreads, E>(fb, fi, nslots * lcap, v, bits);
-      // The fine select over the candidates' key span, floored by the
-      // request's threshold: with a threshold raised by the segments the span
-      // is narrow.  When it is not (short segments) or the boundary bin is
-      // crowded all the same, the candidates' own digit histogram bounds the
-      // K-th largest as a segment's does, and the fine select runs again over
-      // the digits from there up.
-      uint32_t km = 0, kn = 0xFFFFFFFFu;
-#pragma unroll
-      for (int k = 0; k < E; ++k) {
-        km = max(km, (uint32_t)(v[k] >> 32));
-        if (v[k] != 0) kn = min(kn, (uint32_t)(v[k] >> 32));
-      }
-      km = __reduce_max_sync(0xFFFFFFFFu, km);
-      kn = __reduce_min_sync(0xFFFFFFFFu, kn);
-      if (lane_id() == 0) {
-        sc.wsum[threadIdx.x >> 5] = km;
-        sc.wsum[kSelThreads / 32 + (threadIdx.x >> 5)] = kn;
-      }
-      if (threadIdx.x == 0) {
-        *reinterpret_cast<unsigned long long*>(&sc.bcast[0]) = __ldcg(row_thr);
-        *row_thr = 0ull;  // zero for the next call
-      }
-      fine_clear<kSelThreads>(ar);
-      group_sync(kSelThreads);
-      IDX_TRACE(26);
-      km = 0;
-      kn = 0xFFFFFFFFu;
-#pragma unroll
-      for (int w = 0; w < kSelThreads / 32; ++w) {
-        km = max(km, sc.wsum[w]);
-        kn = min(kn, sc.wsum[kSelThreads / 32 + w]);
-      }
-      const uint64_t thr0 = *reinterpret_cast<const unsigned long long*>(&sc.bcast[0]);
-      uint64_t thr = thr0 > ((uint64_t)kn << 32) ? thr0 : ((uint64_t)kn << 32);
-      // (every thread has read wsum and bcast before fine_select's first barrier)
-      if (thr0 != 0)
-        done = fine_select<kSelThreads, E>(v, bits, nkm, thr, km, o.K, ar, out_emit, out_pad);
-      if (!done) {
-        // (the segment's digit histogram is spent: the next segment clears it)
-        hist_clear<kSelThreads>(f.hist, f.hist + kHBins);
-        group_sync(kSelThreads);
-#pragma unroll
-        for (int k = 0; k < E; ++k)
-          if (k < nkm && v[k] >= thr0 && v[k] != 0) {
-            const uint32_t d = (uint32_t)(v[k] >> (32 + kHShift));
-            atomicAdd(&f.hist[d], 1u);
-            atomicAdd(&f.hist[kHBins + (d >> 5)], 1u);
-          }
-        group_sync(kSelThreads);
-        if ((threadIdx.x >> 5) == 0)
-          warp_hist_bounds(f.hist, f.hist + kHBins, (uint32_t)o.K, 0u, sc.bcast);
-        group_sync(kSelThreads);
-        const uint32_t mb0 = sc.bcast[0], mbmax = sc.bcast[1];
-        const uint64_t mlo = (uint64_t)mb0 << (32 + kHShift);
-        thr = thr0 > mlo ? thr0 : mlo;
-        const uint32_t mhi =
-            mbmax + 1 >= (uint32_t)kHBins ? 0xFFFFFFFFu : ((mbmax + 1) << kHShift) - 1u;
-        done = fine_select<kSelThreads, E>(v, bits, nkm, thr, mhi, o.K, ar, out_emit, out_pad);
-      }
-      if (!done) {
-        // a crowded boundary bin (heavy ties): the entries at or above the
-        // threshold go back to the buffer for the exact radix compaction
-        if (threadIdx.x == 0) sc.ctr = 0;
-        group_sync(kSelThreads);
-#pragma unroll
-        for (int k = 0; k < E; ++k)
-          if (k < nkm && v[k] >= thr && v[k] != 0) {
-            const int p = atomicAdd(&sc.ctr, 1);
-            fb[p] = bits[k];
-            fi[p] = ~(uint32_t)v[k];
-          }
-        group_sync(kSelThreads);
-        if (threadIdx.x == 0) {
-          fs.count = sc.ctr;
-          fs.thr = 0ull;
-        }
-        group_sync(kSelThreads);
-        filter_compact<kSelThreads>(fs, fb, fi, o.K, sc);
-        sort_and_write<kSelThreads>(fb, fi, fs.count, o.K, f.sortv, f.sortb, out_i, out_v);
-        done = true;
-      }
-    }
+    if (nslots * lcap <= kFilterCap)
+      done = merge_staged(f, nslots, slot_of, o.cand_bits, o.cand_idx, o.slot_stride, lcap, o.K,
+                          row_thr, f.hist, out_i, out_v);
     if (!done)
       merge_candidates<kSelThreads>(nslots, slot_of, o.cand_bits, o.cand_idx, o.slot_stride,
                                     lcap, o.K, row_thr, fs, f.fbuf, f.fbuf + kFilterCap,
                                     kFilterCap, sc, f.sortv, f.sortb, out_i, out_v);
     IDX_TRACE(16);
   }
+  // every poll of the threshold has landed before the next segment (maybe of
+  // another request) resets s_row, and before the CTA exits
+  cp_async_wait_all();
   group_sync(kSelThreads);
 }
 
@@ -386,19 +431,33 @@ __device__ void fused_finalize(const FusedSel& f, const DecodeArgs& a, int T, in
                                     a.val_out ? a.val_out + orow * a.K : nullptr);
       } else {
         const int64_t slot = (int64_t)(j + b) * T + t;
-        publish_candidates<kSelThreads>(fb, fi, kk, a.K, f.fst[t].thr,
-                                        a.cand_bits + slot * a.slot_stride,
-                                        a.cand_idx + slot * a.slot_stride, a.row_thr + orow);
+        uint32_t* cb = a.cand_bits + slot * a.slot_stride;
+        int32_t* ci = a.cand_idx + slot * a.slot_stride;
+        publish_candidates<kSelThreads>(fb, fi, kk, a.K, f.fst[t].thr, cb, ci, a.row_thr + orow);
+        // padded to a multiple of 4 entries for the staged merge's 16-byte copies
+        for (int p = a.K + (int)threadIdx.x; p < ((a.K + 3) & ~3); p += kSelThreads) {
+          cb[p] = kNegInfBits;
+          ci[p] = -1;
+        }
       }
     }
     if (j0 != j1 && arrive_last<kSelThreads>(a.arrive + b, j1 - j0 + 1, f.s_flag)) {
+      const int nslots = j1 - j0 + 1, lcap = (a.K + 3) & ~3;
       for (int t = 0; t < T; ++t) {
         const int64_t orow = (int64_t)b * T + t;
-        merge_candidates<kSelThreads>(
-            j1 - j0 + 1, [=](int i) { return (int64_t)(j0 + i + b) * T + t; }, a.cand_bits,
-            a.cand_idx, a.slot_stride, a.K, a.K, a.row_thr + orow, f.fst[0], f.fbuf,
-            f.fbuf + kFilterCap, kFilterCap, sc, f.sortv, f.sortb, a.idx_out + orow * a.K,
-            a.val_out ? a.val_out + orow * a.K : nullptr);
+        auto slot_of = [=](int i) { return (int64_t)(j0 + i + b) * T + t; };
+        int32_t* out_i = a.idx_out + orow * a.K;
+        float* out_v = a.val_out ? a.val_out + orow * a.K : nullptr;
+        // (every filter of the CTA is spent: the whole buffer stages the lists)
+        if (nslots * lcap <= kFilterCap)
+          merge_staged(f, nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride, lcap, a.K,
+                       a.row_thr + orow, nullptr, out_i, out_v);
+        else
+          merge_candidates<kSelThreads>(nslots, slot_of, a.cand_bits, a.cand_idx, a.slot_stride,
+                                        a.K, a.K, a.row_thr + orow, f.fst[0], f.fbuf,
+                                        f.fbuf + kFilterCap, kFilterCap, sc, f.sortv, f.sortb,
+                                        out_i, out_v);
+        group_sync(kSelThreads);
       }
     }
   }
