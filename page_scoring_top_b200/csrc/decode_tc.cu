@@ -73,7 +73,10 @@ struct TcLayout {
 __host__ __device__ inline TcLayout tc_layout(bool fused, int D, int T, int Q) {
   TcLayout L;
   L.np = ((T * Q + 15) / 16) * 16;
-  L.cap = fused ? fused_cap(T) : 0;
+  // multi-token rows (no digit histogram) get twice the buffer: their
+  // compactions, which raise the thresholds, come half as often
+  const int bufs = (fused && T > 1) ? 2 : 1;
+  L.cap = fused ? fused_cap(T, bufs) : 0;
   size_t o = 0;
   L.bars = o;  // full[8], empty[8], acc_full[4], acc_empty[4], q_free
   o += 256;
@@ -82,7 +85,7 @@ __host__ __device__ inline TcLayout tc_layout(bool fused, int D, int T, int Q) {
   L.off = o;
   o += al16((size_t)(kDecodeMaxB + 2) * 4);  // prefix sums + the longest length
   L.fbuf = o;
-  o += fused ? (size_t)kFilterCap * 8 : 0;
+  o += fused ? (size_t)bufs * kFilterCap * 8 : 0;
   L.fstate = o;
   o += fused ? al16(sizeof(FilterState) * kMaxFusedT) : 0;
   L.scratch = o;
