@@ -69,7 +69,7 @@ __device__ __forceinline__ void fused_offer(const FusedSel& f, int t, uint32_t b
     filter_offer_h(f.fst[0], f.fbuf, f.fbuf + f.cap, f.hist, f.hist + kHBins, bits, index, valid);
   } else {
     uint32_t* fb = f.fbuf + t * 2 * f.cap;
-    filter_offer(f.fst[t], fb, fb + f.cap, bits, index, valid);
+    filter_offer_lane(f.fst[t], fb, fb + f.cap, bits, index, valid);
   }
 }
 

@@ -164,6 +164,20 @@ __device__ __forceinline__ void filter_offer(FilterState& fs, uint32_t* fb, uint
   }
 }
 
+// filter_offer without the warp vote: each lane that beats the threshold
+// claims its own slot.  Cheaper once the threshold rejects most offers (no
+// warp-wide step for the lanes that append nothing); lanes need not call it
+// together.
+__device__ __forceinline__ void filter_offer_lane(FilterState& fs, uint32_t* fb, uint32_t* fi,
+                                                  uint32_t bits, uint32_t index, bool valid) {
+  const uint64_t v = valid ? rank_value(bits, index) : 0ull;
+  if (v > fs.thr) {
+    const int pos = atomicAdd(&fs.count, 1);
+    fb[pos] = bits;
+    fi[pos] = index;
+  }
+}
+
 // Keep only the top K of the buffer (all NT threads; every offer made before
 // the call must be complete, i.e. the caller syncs the group first).
 template <int NT>
