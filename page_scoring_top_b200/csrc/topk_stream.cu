@@ -331,32 +331,37 @@ __global__ void __launch_bounds__(kTsThreads, 1) topk_stream_kernel(const TopkSt
             }
           }
           if (first) {
-            // A starting threshold before the first offer: cut the stage into
-            // at least K groups (gp groups of 32 / gp scores a thread); every
-            // group's maximum is a distinct score, so the smallest group
-            // maximum is <= the segment's K-th largest.  Without it the
-            // first stage would fill the buffer and force a compaction.
-            const int gp = a.K <= 256 ? 1 : a.K <= 512 ? 2 : a.K <= 1024 ? 4 : 8;
-            uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+            // A starting threshold before the first offer: the digit of the
+            // stage's K-th largest score, from the stage's own digit histogram
+            // (counted into the filter's, still empty, then cleared again).
+            // Every score of the stage's top K is at or above that digit's
+            // floor, so the floor is <= the segment's K-th largest.  Without
+            // it the first stage would fill the buffer and force a compaction.
+            uint32_t* hh = fsel.hist;
+            uint32_t* hc = fsel.hist + kHBins;
 #pragma unroll
             for (int r = 0; r < kTsStage / kTsRound; ++r) {
-              gmax = max(gmax, max(max(order_key(__float_as_uint(x[r].x)),
-                                       order_key(__float_as_uint(x[r].y))),
-                                   max(order_key(__float_as_uint(x[r].z)),
-                                       order_key(__float_as_uint(x[r].w)))));
-              // a group ends every 8 / gp rounds
-              if (((r + 1) * gp) % (kTsStage / kTsRound) == 0) {
-                gmin = min(gmin, gmax);
-                gmax = 0u;
-              }
-            }
-            gmin = __reduce_min_sync(0xFFFFFFFFu, gmin);
-            if (lane == 0) s_wsum[warp] = gmin;
-            group_sync(kTsConsumers);
+              const uint32_t kk[4] = {order_key(__float_as_uint(x[r].x)), order_key(__float_as_uint(x[r].y)),
+                                      order_key(__float_as_uint(x[r].z)), order_key(__float_as_uint(x[r].w))};
 #pragma unroll
-            for (int w = 0; w < kTsConsumerWarps; ++w) gmin = min(gmin, s_wsum[w]);
-            if (gmin != 0u) {  // every group holds a valid score
-              const unsigned long long t = ((unsigned long long)gmin << 32) - 1ull;
+              for (int k = 0; k < 4; ++k)
+                if (kk[k] != 0u && (r * kTsConsumers + tid) * 4 + k < cnt) {
+                  const uint32_t d = kk[k] >> kHShift;
+                  atomicAdd(&hh[d], 1u);
+                  atomicAdd(&hc[d >> 5], 1u);
+                }
+            }
+            group_sync(kTsConsumers);
+            if (warp == 0) {
+              const uint32_t bfl = hist_floor_warp(hh, hc, (uint32_t)a.K);
+              if (lane == 0) s_wsum[0] = bfl;
+            }
+            group_sync(kTsConsumers);
+            const uint32_t bfl = s_wsum[0];
+            hist_clear<kTsConsumers>(hh, hc);
+            group_sync(kTsConsumers);
+            if (bfl != 0u) {
+              const unsigned long long t = ((unsigned long long)bfl << (32 + kHShift)) - 1ull;
               tf = thr_key_float(t);
               if (tid == 0 && t > fs.thr) fs.thr = t;
             }
