@@ -330,13 +330,14 @@ __global__ void __launch_bounds__(kTsThreads, 1) topk_stream_kernel(const TopkSt
                                  __uint_as_float(w[2]), __uint_as_float(w[3]));
             }
           }
-          if (first) {
-            // A starting threshold before the first offer: the digit of the
-            // stage's K-th largest score, from the stage's own digit histogram
-            // (counted into the filter's, still empty, then cleared again).
-            // Every score of the stage's top K is at or above that digit's
-            // floor, so the floor is <= the segment's K-th largest.  Without
-            // it the first stage would fill the buffer and force a compaction.
+          if (first && n > kTsStage) {
+            // A segment of several stages starts from a threshold before its
+            // first offer: the digit of the first stage's K-th largest score,
+            // from the stage's own digit histogram (counted into the filter's,
+            // still empty, then cleared again).  Every score of the stage's
+            // top K is at or above that digit's floor, so the floor is <= the
+            // segment's K-th largest.  Without it the first stages would fill
+            // the buffer and force compactions.
             uint32_t* hh = fsel.hist;
             uint32_t* hc = fsel.hist + kHBins;
 #pragma unroll
@@ -362,6 +363,37 @@ __global__ void __launch_bounds__(kTsThreads, 1) topk_stream_kernel(const TopkSt
             group_sync(kTsConsumers);
             if (bfl != 0u) {
               const unsigned long long t = ((unsigned long long)bfl << (32 + kHShift)) - 1ull;
+              tf = thr_key_float(t);
+              if (tid == 0 && t > fs.thr) fs.thr = t;
+            }
+            first = false;
+          } else if (first) {
+            // A one-stage segment takes a cheaper starting threshold: cut the
+            // stage into at least K groups (gp groups of 32 / gp scores a thread); every
+            // group's maximum is a distinct score, so the smallest group
+            // maximum is <= the segment's K-th largest.  Without it the
+            // first stage would fill the buffer and force a compaction.
+            const int gp = a.K <= 256 ? 1 : a.K <= 512 ? 2 : a.K <= 1024 ? 4 : 8;
+            uint32_t gmin = 0xFFFFFFFFu, gmax = 0u;
+#pragma unroll
+            for (int r = 0; r < kTsStage / kTsRound; ++r) {
+              gmax = max(gmax, max(max(order_key(__float_as_uint(x[r].x)),
+                                       order_key(__float_as_uint(x[r].y))),
+                                   max(order_key(__float_as_uint(x[r].z)),
+                                       order_key(__float_as_uint(x[r].w)))));
+              // a group ends every 8 / gp rounds
+              if (((r + 1) * gp) % (kTsStage / kTsRound) == 0) {
+                gmin = min(gmin, gmax);
+                gmax = 0u;
+              }
+            }
+            gmin = __reduce_min_sync(0xFFFFFFFFu, gmin);
+            if (lane == 0) s_wsum[warp] = gmin;
+            group_sync(kTsConsumers);
+#pragma unroll
+            for (int w = 0; w < kTsConsumerWarps; ++w) gmin = min(gmin, s_wsum[w]);
+            if (gmin != 0u) {  // every group holds a valid score
+              const unsigned long long t = ((unsigned long long)gmin << 32) - 1ull;
               tf = thr_key_float(t);
               if (tid == 0 && t > fs.thr) fs.thr = t;
             }
