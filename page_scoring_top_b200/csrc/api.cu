@@ -80,12 +80,11 @@ int status_of(cudaError_t e) { return e == cudaSuccess ? IDX_OK : IDX_ECUDA; }
 
 int run_topk(idx_ctx* ctx, const float* scores, const int32_t* lengths, int len_div, int rows,
              int N, int64_t lds, int K, int32_t* idx_out, float* val_out, cudaStream_t stream) {
-  if (idx::topk_stream_supported(scores, lds)) {
+  if (idx::topk_stream_supported(scores, lds) && idx::topk_stream_max_rows(N) >= len_div) {
     // the streamed kernel, in blocks of rows; its candidate slots are the
     // fused path's (chunk + row per launch)
     // (a block is a whole number of length groups: rows r use lengths[r / len_div])
-    const int rmax = std::max(1, idx::topk_stream_max_rows() / len_div) * len_div;
-    if (rmax > idx::topk_stream_max_rows()) return IDX_EUNSUPPORTED;
+    const int rmax = (idx::topk_stream_max_rows(N) / len_div) * len_div;
     for (int r0 = 0; r0 < rows; r0 += rmax) {
       const int nr = std::min(rmax, rows - r0);
       if (idx::topk_stream_slots(nr, ctx->num_sms) > ctx->fused_slots) return IDX_ENOWORKSPACE;

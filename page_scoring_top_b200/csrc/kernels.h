@@ -33,7 +33,9 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t stream);
 
 // Streamed top-K (topk_stream.cu): one persistent CTA per SM over the rows laid
 // end to end.  Needs 16-byte aligned scores and lds % 4 == 0; at most
-// topk_stream_max_rows() rows per launch; candidate slots (chunk + row) of
+// topk_stream_max_rows(N) rows of N entries per launch (the entries of a
+// launch, with their per-row charges, are counted in 32 bits; 0 when even one
+// row does not fit); candidate slots (chunk + row) of
 // slot_stride entries, and per-row thresholds and arrival counters that are
 // zero between calls.
 struct TopkStreamArgs {
@@ -54,7 +56,7 @@ struct TopkStreamArgs {
 };
 bool topk_stream_supported(const float* scores, int64_t lds);
 int64_t topk_stream_slots(int rows, int num_sms);
-int topk_stream_max_rows();
+int topk_stream_max_rows(int N);
 cudaError_t launch_topk_stream(const TopkStreamArgs& a, int num_sms, cudaStream_t stream);
 
 // ---------------------------------------------------------------- decode score / fused select

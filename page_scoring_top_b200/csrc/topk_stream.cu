@@ -44,7 +44,7 @@ constexpr int kTsStage = 8192;  // scores per stage (32 KB)
 constexpr int kTsStages = 4;
 constexpr int kTsLanes = 4;       // producer lanes
 constexpr int kTsRound = kTsConsumers * 4;  // scores per offer round (16 bytes a thread)
-constexpr int kTsRowCharge = 16384;  // virtual scores charged per row (a segment-end select)
+constexpr int kTsRowCharge = 49152;  // virtual scores charged per row (a segment-end select and merge)
 constexpr int kTsLMin = kTsStage;    // smallest chunk
 constexpr int kTsMaxRows = kDecodeMaxB;
 constexpr int kTsMaxSegments = 8;    // CTAs per row, for the launch's grid
@@ -473,7 +473,10 @@ int64_t topk_stream_slots(int rows, int num_sms) {
   return (int64_t)num_sms + 1 + (rows < kTsMaxRows ? rows : kTsMaxRows);
 }
 
-int topk_stream_max_rows() { return kTsMaxRows; }
+int topk_stream_max_rows(int N) {
+  const int64_t fit = (int64_t)INT32_MAX / ((int64_t)N + kTsRowCharge);
+  return fit < kTsMaxRows ? (int)fit : kTsMaxRows;
+}
 
 cudaError_t launch_topk_stream(const TopkStreamArgs& a, int num_sms, cudaStream_t stream) {
   const TsLayout L = ts_layout();
