@@ -23,8 +23,9 @@ static_assert(2 * (kSelThreads / 32) <= 32, "per-warp key maxima and minima fit 
 constexpr int kMaxFusedT = 4;
 // Virtual pages charged per request in fused mode: about what a segment-end
 // select step costs in streaming time (a few microseconds at one SM's share
-// of HBM bandwidth, minus what the stage ring absorbs).
-constexpr int kSegmentPages = 896;
+// of HBM bandwidth, minus what the stage ring absorbs; measured best among
+// 256 .. 2304 on the decode workloads).
+constexpr int kSegmentPages = 512;
 
 // Shared-memory state of the fused select (pointers into the kernel's layout).
 struct FusedSel {
