@@ -309,7 +309,11 @@ __global__ void __launch_bounds__(kTsThreads, 1) topk_stream_kernel(const TopkSt
         // 16-byte read, three max and one compare; the few that pass take
         // the exact offer.  The threshold is read once a stage (a stale one
         // is lower, so it only lets more through).
-        float tf = thr_key_float(*reinterpret_cast<volatile unsigned long long*>(&fs.thr));
+        const unsigned long long thr_now = *reinterpret_cast<volatile unsigned long long*>(&fs.thr);
+        float tf = thr_key_float(thr_now);
+        // a score equal to tf (its key the threshold's key half) passes only
+        // below this index (ties go to the lower index)
+        uint32_t ilim = ~(uint32_t)thr_now;
         {
           // All 32 scores first (a bit per score that may pass), then the
           // exact offers of the few that may: a warp walks the slow path
@@ -364,6 +368,7 @@ __global__ void __launch_bounds__(kTsThreads, 1) topk_stream_kernel(const TopkSt
             if (bfl != 0u) {
               const unsigned long long t = ((unsigned long long)bfl << (32 + kHShift)) - 1ull;
               tf = thr_key_float(t);
+              ilim = 0u;
               if (tid == 0 && t > fs.thr) fs.thr = t;
             }
             first = false;
@@ -395,16 +400,27 @@ __global__ void __launch_bounds__(kTsThreads, 1) topk_stream_kernel(const TopkSt
             if (gmin != 0u) {  // every group holds a valid score
               const unsigned long long t = ((unsigned long long)gmin << 32) - 1ull;
               tf = thr_key_float(t);
+              ilim = 0u;
               if (tid == 0 && t > fs.thr) fs.thr = t;
             }
             first = false;
           }
           uint32_t maybe = 0;
+          if ((uint32_t)o >= ilim) {
+            // no score of the stage that ties the threshold's key can pass
+            // (heavy ties would otherwise all take the exact offer)
 #pragma unroll
-          for (int r = 0; r < kTsStage / kTsRound; ++r)
-            maybe |= ((uint32_t)(x[r].x >= tf) | (uint32_t)(x[r].y >= tf) << 1 |
-                      (uint32_t)(x[r].z >= tf) << 2 | (uint32_t)(x[r].w >= tf) << 3)
-                     << (4 * r);
+            for (int r = 0; r < kTsStage / kTsRound; ++r)
+              maybe |= ((uint32_t)(x[r].x > tf) | (uint32_t)(x[r].y > tf) << 1 |
+                        (uint32_t)(x[r].z > tf) << 2 | (uint32_t)(x[r].w > tf) << 3)
+                       << (4 * r);
+          } else {
+#pragma unroll
+            for (int r = 0; r < kTsStage / kTsRound; ++r)
+              maybe |= ((uint32_t)(x[r].x >= tf) | (uint32_t)(x[r].y >= tf) << 1 |
+                        (uint32_t)(x[r].z >= tf) << 2 | (uint32_t)(x[r].w >= tf) << 3)
+                       << (4 * r);
+          }
           if (cnt < kTsStage) {  // only positions that hold a score
 #pragma unroll
             for (int r = 0; r < kTsStage / kTsRound; ++r)
